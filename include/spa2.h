@@ -1,0 +1,200 @@
+/*
+ * spa2.h -- C ABI of libspa2.so: hybrid Top-k + Top-p block-sparse attention
+ * (SpargeAttention2) on NVIDIA B200 (sm_100a).
+ *
+ * The operations are those of arXiv 2602.13515, "SpargeAttention2: Trainable
+ * Sparse Attention via Hybrid Top-k+Top-p Masking and Distillation
+ * Fine-Tuning", as summarised on
+ *   - paper.rainbus.top (SpargeAttention2 summary), sections 前置知识
+ *     (sparse / Top-k / Top-p / block-sparse attention), 方法步骤详情 (method
+ *     steps 1-4) and 技术新颖性 (the union formula);
+ *   - gist.science (same title), section 2A "Hybrid Top-k + Top-p Masking"
+ *     and 2C "Efficient Kernel Implementation";
+ *   - chatpaper.ai abstract ("efficient trainable sparse attention
+ *     implementation": forward and backward).
+ *
+ * Conventions shared by every entry point
+ * ----------------------------------------
+ * Tensors. Q, K, V, O, dO, dQ, dK, dV are contiguous [B, H, N, d] bf16 in
+ *   device memory, 16-byte aligned. LSE is [B, H, N] fp32 (natural log of the
+ *   row sum of exp(scaled logits)). Block counts: T_m = ceil(N / bq),
+ *   T_n = ceil(N / bkv); the last block of a ragged N is partial.
+ * Supported set. d in {64, 128}; (bq, bkv) = (128, 64); N >= 1; B, H >= 1;
+ *   0 <= k_frac <= 1, 0 <= p_frac <= 1. Anything else returns
+ *   SPA2_ERR_UNSUPPORTED (or SPA2_ERR_INVALID_ARG for nonsense such as a null
+ *   pointer or a negative size) and launches nothing.
+ * Ownership. The caller allocates and owns every buffer, including the
+ *   workspace `ws` (size from spa2_workspace_bytes, 256-byte aligned). The
+ *   library never allocates or frees device memory and keeps no pointer
+ *   after a call returns.
+ * Streams. All work is enqueued asynchronously on `stream` (NULL = the
+ *   legacy default stream); a call returns once its kernels are enqueued.
+ * Errors. Argument errors are returned synchronously before anything is
+ *   launched. A failed launch returns SPA2_ERR_CUDA. Faults detected on the
+ *   device (a bounded wait that ran out, an index outside its buffer) are
+ *   recorded in the status word (the first 4 bytes of `ws`, cleared at the
+ *   start of every call) and read back by spa2_stream_status. The library
+ *   never aborts, asserts or traps.
+ */
+#ifndef SPA2_H
+#define SPA2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define SPA2_API __attribute__((visibility("default")))
+#else
+#define SPA2_API
+#endif
+
+typedef struct CUstream_st* spa2_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  SPA2_OK = 0,
+  SPA2_ERR_INVALID_ARG = 1,    /* null pointer, negative size, misaligned pointer */
+  SPA2_ERR_UNSUPPORTED = 2,    /* valid but outside the supported set above */
+  SPA2_ERR_CUDA = 3,           /* a CUDA runtime / driver call failed */
+  SPA2_ERR_DEVICE_TIMEOUT = 4, /* a device-side bounded wait ran out */
+  SPA2_ERR_WORKSPACE = 5,      /* ws is NULL or smaller than spa2_workspace_bytes */
+  SPA2_ERR_DEVICE_BOUNDS = 6   /* a device-side index check failed (bad mask) */
+} spa2_status;
+
+/*
+ * Block mask in compressed form. All pointers are device pointers owned by
+ * the caller. Kept ids of a row (column) are listed in ascending order; only
+ * the first row_cnt (col_cnt) entries of a row (column) are meaningful.
+ *   row_cnt [B, H, T_m]       int32  kept kv-blocks per q-block (>= 1)
+ *   row_idx [B, H, T_m, T_n]  int32  kept kv-block ids of each q-block (CSR)
+ *   col_cnt [B, H, T_n]       int32  q-blocks keeping each kv-block
+ *   col_idx [B, H, T_n, T_m]  int32  those q-block ids (CSC)
+ *   pbar    [B, H, T_m, T_n]  fp32   pooled attention P-bar, or NULL
+ *   bitmap  [B, H, T_m, T_n]  uint8  1 = kept, or NULL
+ * spa2_sparse_attn_fwd reads row_cnt/row_idx; spa2_sparse_attn_bwd reads
+ * col_cnt/col_idx; the mask builders write all non-NULL fields (col_* may be
+ * NULL when no backward pass will follow).
+ */
+typedef struct {
+  int32_t* row_cnt;
+  int32_t* row_idx;
+  int32_t* col_cnt;
+  int32_t* col_idx;
+  float* pbar;
+  uint8_t* bitmap;
+} spa2_mask;
+
+enum { SPA2_OP_MASK = 0, SPA2_OP_FWD = 1, SPA2_OP_BWD = 2, SPA2_OP_SELECT = 3 };
+
+/* ABI version of this header (bumped on any incompatible change). */
+#define SPA2_ABI_VERSION 1
+SPA2_API int spa2_abi_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+SPA2_API const char* spa2_status_string(spa2_status s);
+
+/*
+ * Workspace bytes needed by `op` (SPA2_OP_*) for this shape; 0 for an
+ * unsupported shape. For SPA2_OP_SELECT the arguments are read as
+ * (B, H, T_m, T_n) = (B, H, N, d) and bq, bkv are ignored. Every workspace
+ * starts with the 256-byte status block.
+ */
+SPA2_API size_t spa2_workspace_bytes(int op, int B, int H, int N, int d, int bq, int bkv);
+
+/*
+ * Steps 1-3 of the method (paper.rainbus.top, 方法步骤详情, steps 1-3):
+ *   1. partition Q into T_m blocks of bq rows, K into T_n blocks of bkv rows;
+ *   2. pool each block to its mean row (fp32) and form the pooled attention
+ *      P-bar = softmax(pool(Q) pool(K)^T / sqrt(d)), row by row;
+ *   3. keep block j of row i iff j is in Top-k(P-bar_i, k_frac) or in
+ *      Top-p(P-bar_i, p_frac) (union; 技术新颖性 formula).
+ * Selection rule (exact, deterministic): rank the row by (P-bar descending,
+ * block id ascending); K = clamp(floor(k_frac * T_n + 0.5), 1, T_n) in double;
+ * Top-p keeps rank r while floor(2^32 * mass of ranks < r) < floor(2^32 *
+ * p_frac), masses quantised per block as floor(2^32 * P-bar_j) (the first
+ * prefix whose mass reaches p, sink row example of 研究动机); the union is the
+ * first max(K, R) ranks. Writes every non-NULL field of *out.
+ *   q, k : [B, H, N, d] bf16 device pointers (read only)
+ *   out  : host pointer to a spa2_mask of device pointers (see above)
+ *   ws   : device workspace of spa2_workspace_bytes(SPA2_OP_MASK, ...) bytes
+ */
+SPA2_API spa2_status spa2_block_mask(const void* q, const void* k, int B, int H, int N, int d, int bq, int bkv,
+                            float k_frac, float p_frac, const spa2_mask* out, void* ws, size_t ws_bytes,
+                            spa2_stream_t stream);
+
+/*
+ * Step 3 alone on a caller-given P-bar (parity checks of the selection rule,
+ * and masks computed elsewhere). Same rule and outputs as spa2_block_mask;
+ * out->pbar is ignored. pbar entries must be finite and in [0, 1].
+ *   pbar : [B, H, T_m, T_n] fp32 device pointer
+ *   ws   : spa2_workspace_bytes(SPA2_OP_SELECT, B, H, T_m, T_n, 0, 0) bytes
+ */
+SPA2_API spa2_status spa2_select_blocks(const float* pbar, int B, int H, int Tm, int Tn, float k_frac, float p_frac,
+                               const spa2_mask* out, void* ws, size_t ws_bytes, spa2_stream_t stream);
+
+/*
+ * Step 4 forward (paper.rainbus.top, 方法步骤详情 step 4 and 前置知识 "稀疏注意力",
+ * "块稀疏注意力"; gist.science 2C): for every q-block i and every kept kv-block j
+ * of row i, S_ij = Q_i K_j^T * softmax_scale, online softmax, O_i += P_ij V_j;
+ * masked (i, j) tiles are skipped entirely. No causal mask.
+ *   q, k, v       : [B, H, N, d] bf16 device pointers (read only)
+ *   mask          : host pointer to a spa2_mask; row_cnt/row_idx are read
+ *   softmax_scale : logit scale; 0 means 1/sqrt(d)
+ *   o             : [B, H, N, d] bf16 device output
+ *   lse           : [B, H, N] fp32 device output (natural-log LSE)
+ *   ws            : spa2_workspace_bytes(SPA2_OP_FWD, ...) bytes
+ */
+SPA2_API spa2_status spa2_sparse_attn_fwd(const void* q, const void* k, const void* v, int B, int H, int N, int d, int bq,
+                                 int bkv, const spa2_mask* mask, float softmax_scale, void* o, float* lse, void* ws,
+                                 size_t ws_bytes, spa2_stream_t stream);
+
+/*
+ * Step 4 backward through the same block mask (the trainable part;
+ * chatpaper.ai abstract (ii)): with P = exp(S - LSE) on kept tiles,
+ *   dV_j = sum_i P_ij^T dO_i,  dP_ij = dO_i V_j^T,  D_i = rowsum(dO_i * O_i),
+ *   dS_ij = P_ij * (dP_ij - D_i),  dQ_i = sum_j dS_ij K_j * scale,
+ *   dK_j = sum_i dS_ij^T Q_i * scale.
+ * The mask is held constant (no gradient through pooling or selection).
+ *   q, k, v, o, dout : [B, H, N, d] bf16 device pointers (read only); o and
+ *                      lse are the forward outputs for the same mask
+ *   lse              : [B, H, N] fp32 device pointer
+ *   mask             : host pointer to a spa2_mask; col_cnt/col_idx are read
+ *   dq, dk, dv       : [B, H, N, d] bf16 device outputs
+ *   ws               : spa2_workspace_bytes(SPA2_OP_BWD, ...) bytes (holds the
+ *                      fp32 dQ accumulator and D)
+ */
+SPA2_API spa2_status spa2_sparse_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                                 const void* dout, int B, int H, int N, int d, int bq, int bkv, const spa2_mask* mask,
+                                 float softmax_scale, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
+                                 spa2_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the status word at the start
+ * of `ws`. Returns SPA2_OK, the first device-side error recorded since the
+ * word was last cleared, or SPA2_ERR_CUDA if the stream itself failed.
+ */
+SPA2_API spa2_status spa2_stream_status(void* ws, spa2_stream_t stream);
+
+/*
+ * Fault-path testing. Sets the time limit, in nanoseconds, of every bounded
+ * device-side wait launched afterwards by this process (default 2e9 = 2 s;
+ * limit <= 0 restores the default). Returns SPA2_OK.
+ */
+SPA2_API spa2_status spa2_debug_set_wait_limit_ns(long long limit);
+
+/*
+ * Fault-path testing. Launches one CTA that waits on an mbarrier nothing
+ * arrives on, bounded by the current wait limit; the wait runs out, the
+ * kernel records SPA2_ERR_DEVICE_TIMEOUT in the status word of `ws` (>= 256
+ * bytes) and returns normally, leaving the context usable.
+ */
+SPA2_API spa2_status spa2_debug_timeout_probe(void* ws, size_t ws_bytes, spa2_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPA2_H */

@@ -1,0 +1,52 @@
+"""Shared comparison helpers for the GPU parity tests."""
+
+import numpy as np
+
+# BASELINE tolerance for attention outputs and gradients (bf16 inputs, fp32
+# accumulation): max-abs 2e-2 and relative L1 1e-2, element by element.
+MAX_ABS = 2e-2
+REL_L1 = 1e-2
+
+
+def f64(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def assert_close(actual, expected, what, max_abs=MAX_ABS, rel_l1=REL_L1):
+    a = np.asarray(actual, dtype=np.float64)
+    e = np.asarray(expected, dtype=np.float64)
+    assert a.shape == e.shape, (what, a.shape, e.shape)
+    assert np.isfinite(a).all(), f"{what}: non-finite values"
+    err = np.abs(a - e)
+    ma = float(err.max()) if err.size else 0.0
+    rl1 = float(err.sum() / max(np.abs(e).sum(), 1e-300))
+    assert ma <= max_abs and rl1 <= rel_l1, f"{what}: max_abs={ma:.3e} (<= {max_abs}) rel_l1={rl1:.3e} (<= {rel_l1})"
+    return ma, rl1
+
+
+def csr_to_dense(row_cnt, row_idx, Tn):
+    """bool [.., Tm, Tn] from CSR numpy arrays; checks ids ascending and in range."""
+    cnt = np.asarray(row_cnt)
+    idx = np.asarray(row_idx)
+    out = np.zeros(cnt.shape + (Tn,), dtype=bool)
+    for pos in np.ndindex(cnt.shape):
+        n = int(cnt[pos])
+        ids = idx[pos][:n]
+        assert 1 <= n <= Tn
+        assert (np.diff(ids) > 0).all() and ids.min() >= 0 and ids.max() < Tn
+        out[pos][ids] = True
+    return out
+
+
+def csc_to_dense(col_cnt, col_idx, Tm):
+    cnt = np.asarray(col_cnt)
+    idx = np.asarray(col_idx)
+    out = np.zeros(cnt.shape + (Tm,), dtype=bool)
+    for pos in np.ndindex(cnt.shape):
+        n = int(cnt[pos])
+        ids = idx[pos][:n]
+        assert 0 <= n <= Tm
+        if n:
+            assert (np.diff(ids) > 0).all() and ids.min() >= 0 and ids.max() < Tm
+        out[pos][ids] = True
+    return np.swapaxes(out, -1, -2)

@@ -1,0 +1,148 @@
+"""GPU parity of the block-sparse attention forward (O, LSE) and backward
+(dQ, dK, dV) against the float64 oracle, under the GPU's own block mask,
+through the C ABI. Tolerance: max-abs 2e-2 and relative L1 1e-2."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests._parity import assert_close, csr_to_dense, f64
+from trainable_block_sparse_pooled_b200 import binding as b
+from trainable_block_sparse_pooled_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(q, k, v, kf, pf, dout=None, mask=None):
+    B, H, N, d = q.shape
+    s = b.Spa2(B, H, N, d)
+    m = s.block_mask(q, k, kf, pf) if mask is None else mask
+    o, lse = s.fwd(q, k, v, m)
+    grads = None
+    if dout is not None:
+        grads = s.bwd(q, k, v, o, lse, dout, m)
+    s.check()
+    dense = csr_to_dense(m.row_cnt.cpu().numpy(), m.row_idx.cpu().numpy(), s.Tn)
+    return s, m, dense, o, lse, grads
+
+
+def _check_fwd(q, k, v, dense, o, lse):
+    O, LSE = oracle.masked_attn_fwd(f64(q), f64(k), f64(v), dense, 128, 64)
+    assert_close(f64(o), O, "O")
+    assert_close(lse.cpu().numpy(), LSE, "LSE")
+
+
+def _check_bwd(q, k, v, dense, dout, grads):
+    dQ, dK, dV = oracle.masked_attn_bwd(f64(q), f64(k), f64(v), dense, f64(dout), 128, 64)
+    assert_close(f64(grads[0]), dQ, "dQ")
+    assert_close(f64(grads[1]), dK, "dK")
+    assert_close(f64(grads[2]), dV, "dV")
+
+
+def test_pr1_fwd_bwd():
+    """B=1 H=2 N=512 d=64, N(0,1) with 2 sinks, k=20% p=60%, forward + backward."""
+    q, k, v = synth.gaussian_with_sinks(B=1, H=2, N=512, d=64, seed=0, device="cuda")
+    dout = synth.normal_like(q.shape, seed=1, device="cuda")
+    _, _, dense, o, lse, grads = _run(q, k, v, 0.2, 0.6, dout)
+    _check_fwd(q, k, v, dense, o, lse)
+    _check_bwd(q, k, v, dense, dout, grads)
+
+
+@pytest.mark.parametrize("N,d,kf,pf", [(1000, 128, 0.1, 0.5), (1000, 64, 0.2, 0.3), (130, 128, 0.0, 0.7),
+                                       (2049, 128, 0.05, 0.9), (333, 64, 1.0, 0.0)])
+def test_ragged_fwd_bwd(N, d, kf, pf):
+    q, k, v = synth.gaussian_with_sinks(B=2, H=2, N=N, d=d, seed=N, device="cuda")
+    dout = synth.normal_like(q.shape, seed=N + 1, device="cuda")
+    _, _, dense, o, lse, grads = _run(q, k, v, kf, pf, dout)
+    _check_fwd(q, k, v, dense, o, lse)
+    _check_bwd(q, k, v, dense, dout, grads)
+
+
+def test_dense_k100_equals_full_attention():
+    q, k, v = synth.gaussian_with_sinks(B=1, H=2, N=640, d=128, seed=5, device="cuda")
+    _, m, dense, o, lse, _ = _run(q, k, v, 1.0, 0.0)
+    assert dense.all()
+    ref = torch.nn.functional.scaled_dot_product_attention(q.double().cpu(), k.double().cpu(), v.double().cpu())
+    assert_close(f64(o), ref.numpy(), "O vs SDPA")
+
+
+def test_uncovered_kv_block_gets_zero_grads():
+    """A kv-block no q-block keeps: dK = dV = 0 there (CSC column is empty)."""
+    B, H, N, d = 1, 1, 640, 128
+    q, k, v = synth.gaussian_with_sinks(B=B, H=H, N=N, d=d, seed=9, device="cuda")
+    dout = synth.normal_like(q.shape, seed=10, device="cuda")
+    Tm, Tn = b.block_counts(N)
+    rng = np.random.default_rng(0)
+    pbar = rng.dirichlet(np.ones(Tn), size=(B, H, Tm)).astype(np.float32)
+    pbar[..., 3] = 0.0
+    mask = b.select_blocks(torch.tensor(pbar, device="cuda"), 0.2, 0.5)
+    assert int(mask.col_cnt[0, 0, 3]) == 0
+    _, _, dense, o, lse, grads = _run(q, k, v, 0, 0, dout, mask=mask)
+    assert not dense[..., 3].any()
+    assert torch.count_nonzero(grads[1][0, 0, 192:256]) == 0
+    assert torch.count_nonzero(grads[2][0, 0, 192:256]) == 0
+    _check_fwd(q, k, v, dense, o, lse)
+    _check_bwd(q, k, v, dense, dout, grads)
+
+
+def test_forward_is_deterministic():
+    q, k, v = synth.gaussian_with_sinks(B=1, H=4, N=3000, d=128, seed=2, device="cuda")
+    s = b.Spa2(1, 4, 3000, 128)
+    m = s.block_mask(q, k, 0.05, 0.8)
+    o1, l1 = s.fwd(q, k, v, m)
+    o2, l2 = s.fwd(q, k, v, m)
+    s.check()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_mixed_rows_fwd_bwd_small():
+    """Config-3 recipe (near-uniform even q-blocks, +6-logit skewed odd q-blocks,
+    k=5% p=90%) on the 8x32x32 grid, whole heads, forward and backward."""
+    q, k, v = synth.mixed_rows(B=1, H=2, N=8192, d=128, seed=4, device="cuda", grid=(8, 32, 32))
+    dout = synth.normal_like(q.shape, seed=5, device="cuda")
+    _, m, dense, o, lse, grads = _run(q, k, v, 0.05, 0.9, dout)
+    cnt = m.row_cnt.cpu().numpy()[0]
+    assert cnt[:, 0::2].mean() > cnt[:, 1::2].mean()      # uniform rows keep more blocks
+    _check_fwd(q, k, v, dense, o, lse)
+    _check_bwd(q, k, v, dense, dout, grads)
+
+
+@pytest.mark.slow
+def test_wan13b_fwd_sampled_qblocks():
+    """1.3B layer (B1 H12 N32760 d128, smoothed field + 4 sinks) at k=2.5% p=60%:
+    16 seeded q-blocks per head plus the last (120-row) q-block, every head."""
+    q, k, v = synth.smoothed_field(B=1, H=12, N=32760, d=128, seed=1, device="cuda")
+    s, m, dense, o, lse, _ = _run(q, k, v, 0.025, 0.6)
+    rng = np.random.default_rng(0)
+    qf, kf_, vf = f64(q), f64(k), f64(v)
+    o64 = f64(o)
+    l64 = lse.cpu().numpy()
+    for h in range(12):
+        blocks = sorted(set(rng.integers(0, s.Tm - 1, 16).tolist()) | {s.Tm - 1})
+        ref = oracle.masked_attn_fwd_rows(qf, kf_, vf, dense, 128, 64, 1 / np.sqrt(128), 0, h, blocks)
+        for i, (Oi, Li) in ref.items():
+            assert_close(o64[0, h, i * 128:i * 128 + Oi.shape[0]], Oi, f"O h{h} i{i}")
+            assert_close(l64[0, h, i * 128:i * 128 + Oi.shape[0]], Li, f"LSE h{h} i{i}")
+
+
+@pytest.mark.slow
+def test_wan13b_bwd_sampled_blocks():
+    """1.3B shape, mixed rows (config-3 recipe), k=5% p=90%, forward + backward:
+    dQ of 8 sampled q-blocks and dK, dV of 8 sampled kv-blocks (the last, ragged,
+    one included) in heads 0 and 11, against the oracle."""
+    q, k, v = synth.mixed_rows(B=1, H=12, N=32760, d=128, seed=2, device="cuda")
+    dout = synth.normal_like(q.shape, seed=3, device="cuda")
+    s, m, dense, o, lse, grads = _run(q, k, v, 0.05, 0.9, dout)
+    rng = np.random.default_rng(1)
+    qf, kf_, vf, df = f64(q), f64(k), f64(v), f64(dout)
+    dq, dk, dv = (f64(g) for g in grads)
+    for h in (0, 11):
+        qb = sorted(set(rng.integers(0, s.Tm, 8).tolist()))
+        kb = sorted(set(rng.integers(0, s.Tn - 1, 7).tolist()) | {s.Tn - 1})
+        sq, skv = oracle.masked_attn_bwd_blocks(qf, kf_, vf, dense, df, 128, 64, 1 / np.sqrt(128), 0, h, qb, kb)
+        for i, g in sq.items():
+            assert_close(dq[0, h, i * 128:i * 128 + g.shape[0]], g, f"dQ h{h} i{i}")
+        for j, (gk, gv) in skv.items():
+            assert_close(dk[0, h, j * 64:j * 64 + gk.shape[0]], gk, f"dK h{h} j{j}")
+            assert_close(dv[0, h, j * 64:j * 64 + gv.shape[0]], gv, f"dV h{h} j{j}")

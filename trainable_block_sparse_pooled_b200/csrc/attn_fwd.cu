@@ -1,0 +1,320 @@
+// Block-sparse attention forward on sm_100a: step 4 of SpargeAttention2
+// (paper.rainbus.top summary, 方法步骤详情 step 4; 前置知识 "稀疏注意力" and
+// "块稀疏注意力": masked Q_i K_j^T and P_ij V_j tiles are skipped; gist.science 2C).
+//
+// One CTA per (q-block i, head): 128 query rows (b_q = 128) against the kept
+// kv-blocks j (b_kv = 64 rows each) listed in the CSR row of i.
+//
+//   warp 4      TMA producer: Q_i once, then K_j / V_j through a 2-slot ring.
+//   warp 5      MMA issuer (one thread): S = Q K_j^T (SS, M=128 N=64 K=d) into
+//               one of two TMEM S buffers; O += P V_j (TS: P from TMEM,
+//               M=128 N=d K=64). Owns the 256-column TMEM allocation.
+//   warps 0-3   softmax, thread t <-> query row t <-> TMEM lane t: load S,
+//               online max / exp2 / sum in registers, write P (bf16) over the
+//               S buffer, rescale O in TMEM only when the running max grew by
+//               more than 2^8 (lazy rescale), then the epilogue O / l -> bf16
+//               -> smem -> TMA store, and LSE.
+//
+// TMEM columns: [0,64) S/P buffer 0, [64,128) S/P buffer 1, [128,128+d) O.
+// Shared memory: Q 128 x d bf16 (reused as the O staging tile), 2 x (K, V)
+// 64 x d bf16; every tile in 128-byte-swizzled 64-column chunks as TMA writes
+// them. Two CTAs fit on one SM (TMEM 2 x 256 columns, smem 2 x ~97 KB), so one
+// CTA's softmax overlaps the other's MMAs.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace spa2 {
+
+namespace {
+
+template <int D>
+struct FwdSmem {
+  static constexpr int CH = D / 64;  // 64-column chunks per row
+  alignas(1024) uint8_t q[CH][128 * 128];
+  alignas(1024) uint8_t k[2][CH][64 * 128];
+  alignas(1024) uint8_t v[2][CH][64 * 128];
+  uint64_t q_full;
+  uint64_t k_full[2], v_full[2], kv_empty[2];
+  uint64_t s_full[2], p_full[2], o_done, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int epi_ok;
+  int never;  // stays 0: abort flag of the teardown drains
+};
+
+SPA2_DEV bool wait_warp(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
+  const bool ok = wait_bar(bar, parity, w);
+  return __all_sync(0xffffffff, ok);
+}
+
+}  // namespace
+
+template <int D>
+__global__ void __launch_bounds__(192, 2) fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                                     const __grid_constant__ CUtensorMap tm_k,
+                                                     const __grid_constant__ CUtensorMap tm_v,
+                                                     const __grid_constant__ CUtensorMap tm_o,
+                                                     const int* __restrict__ row_cnt, const int* __restrict__ row_idx,
+                                                     float* __restrict__ lse, int N, int Tm, int Tn, float scale_log2,
+                                                     int* status, unsigned long long wait_limit_ns) {
+  constexpr int CH = D / 64;
+  constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, false, false);
+  constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, false, true);
+  constexpr uint32_t Q_BYTES = 128 * D * 2;
+  constexpr uint32_t KV_BYTES = 64 * D * 2;
+
+  extern __shared__ uint8_t smem_raw[];
+  FwdSmem<D>& sm = *reinterpret_cast<FwdSmem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+  const int warp = threadIdx.x >> 5;
+  const uint32_t lane = lane_id();
+  const int i = blockIdx.x;
+  const int bh = blockIdx.y;
+  const long long rowid = (long long)bh * Tm + i;
+
+  if (warp == 5) {
+    tmem_alloc(&sm.tmem_base, 256);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 128) {
+    mbar_init(&sm.q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sm.k_full[s], 1);
+      mbar_init(&sm.v_full[s], 1);
+      mbar_init(&sm.kv_empty[s], 1);
+      mbar_init(&sm.s_full[s], 1);
+      mbar_init(&sm.p_full[s], 128);
+    }
+    mbar_init(&sm.o_done, 1);
+    mbar_init(&sm.drain, 1);
+    sm.abort_flag = 0;
+    sm.epi_ok = 0;
+    sm.never = 0;
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const WaitCtx wc{&sm.abort_flag, status, wait_limit_ns};
+
+  int n = row_cnt[rowid];
+  if (n < 1 || n > Tn) {
+    if (threadIdx.x == 0) report(status, SPA2_ERR_DEVICE_BOUNDS);
+    n = 0;
+  }
+  const int* kv_list = row_idx + rowid * Tn;
+
+  if (warp == 4) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0 && n > 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_expect_tx(&sm.q_full, Q_BYTES);
+      for (int c = 0; c < CH; ++c) tma_load_3d(sm.q[c], &tm_q, &sm.q_full, c * 64, i * 128, bh);
+      int issued = 0;
+      for (int t = 0; t < n; ++t) {
+        const int s = t & 1;
+        if (t >= 2 && !wait_bar(&sm.kv_empty[s], ((t >> 1) - 1) & 1, wc)) break;
+        const int j = kv_list[t];
+        if (j < 0 || j >= Tn) {
+          report(status, SPA2_ERR_DEVICE_BOUNDS);
+          sm.abort_flag = 1;
+          break;
+        }
+        mbar_expect_tx(&sm.k_full[s], KV_BYTES);
+        for (int c = 0; c < CH; ++c) tma_load_3d(sm.k[s][c], &tm_k, &sm.k_full[s], c * 64, j * 64, bh);
+        mbar_expect_tx(&sm.v_full[s], KV_BYTES);
+        for (int c = 0; c < CH; ++c) tma_load_3d(sm.v[s][c], &tm_v, &sm.v_full[s], c * 64, j * 64, bh);
+        issued = t + 1;
+      }
+      // never leave with copies in flight: wait (bounded) for the last loads
+      const WaitCtx drain_wc{&sm.never, nullptr, wait_limit_ns};
+      for (int t = max(0, issued - 2); t < issued; ++t) {
+        wait_bar(&sm.k_full[t & 1], (t >> 1) & 1, drain_wc);
+        wait_bar(&sm.v_full[t & 1], (t >> 1) & 1, drain_wc);
+      }
+      wait_bar(&sm.q_full, 0, drain_wc);
+    }
+  } else if (warp == 5) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0 && n > 0) {
+      const uint32_t tmem_o = tmem + 128;
+      if (wait_bar(&sm.q_full, 0, wc)) {
+        for (int t = 0; t <= n; ++t) {
+          if (t < n) {
+            const int s = t & 1;
+            if (!wait_bar(&sm.k_full[s], (t >> 1) & 1, wc)) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t a = sdesc_sw128(smem_u32(sm.q[kk >> 2]) + (kk & 3) * 32, 16, 1024);
+              const uint64_t b = sdesc_sw128(smem_u32(sm.k[s][kk >> 2]) + (kk & 3) * 32, 16, 1024);
+              mma_ss(tmem + s * 64, a, b, IDESC_S, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(&sm.s_full[s]);
+          }
+          if (t >= 1) {
+            const int u = t - 1, su = u & 1;
+            if (!wait_bar(&sm.p_full[su], (u >> 1) & 1, wc)) break;
+            if (!wait_bar(&sm.v_full[su], (u >> 1) & 1, wc)) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t b = sdesc_sw128(smem_u32(sm.v[su][0]) + kk * 2048, 64 * 128, 1024);
+              mma_ts(tmem_o, tmem + su * 64 + kk * 8, b, IDESC_O, (u > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(&sm.kv_empty[su]);
+            mma_commit(&sm.o_done);
+          }
+        }
+      }
+      // drain: every MMA issued above completes before TMEM is released
+      mma_commit(&sm.drain);
+      const WaitCtx drain_wc{&sm.never, nullptr, wait_limit_ns};
+      wait_bar(&sm.drain, 0, drain_wc);
+    }
+  } else {
+    // ---------------- softmax warps 0-3 ----------------
+    const int r = threadIdx.x;                       // row in the tile == TMEM lane
+    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    float m_use = -INFINITY, l = 0.f;
+    bool ok = n > 0;
+    for (int t = 0; t < n && ok; ++t) {
+      const int s = t & 1;
+      if (!wait_warp(&sm.s_full[s], (t >> 1) & 1, wc)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int j = kv_list[t];
+      const int valid = (j == Tn - 1) ? (N - j * 64) : 64;
+      uint32_t ra[32], rb[32];
+      tmem_ld32(tl + s * 64, ra);
+      tmem_ld32(tl + s * 64 + 32, rb);
+      tmem_wait_ld();
+      float mx = -INFINITY;
+      if (valid >= 64) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) mx = fmaxf(mx, fmaxf(__uint_as_float(ra[c]), __uint_as_float(rb[c])));
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          if (c >= valid) ra[c] = __float_as_uint(-INFINITY);
+          if (c + 32 >= valid) rb[c] = __float_as_uint(-INFINITY);
+          mx = fmaxf(mx, fmaxf(__uint_as_float(ra[c]), __uint_as_float(rb[c])));
+        }
+      }
+      const float m_new = fmaxf(m_use, mx * scale_log2);
+      float alpha = 1.f;
+      bool rescale = false;
+      if (m_use == -INFINITY) {
+        m_use = m_new;
+      } else if (m_new > m_use + 8.0f) {
+        alpha = fast_exp2(m_use - m_new);
+        m_use = m_new;
+        l *= alpha;
+        rescale = true;
+      }
+      const float neg_m = -m_use;
+      uint32_t pk[32];
+      float rs = 0.f;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const float p0 = fast_exp2(fmaf(__uint_as_float(ra[2 * c]), scale_log2, neg_m));
+        const float p1 = fast_exp2(fmaf(__uint_as_float(ra[2 * c + 1]), scale_log2, neg_m));
+        const float p2 = fast_exp2(fmaf(__uint_as_float(rb[2 * c]), scale_log2, neg_m));
+        const float p3 = fast_exp2(fmaf(__uint_as_float(rb[2 * c + 1]), scale_log2, neg_m));
+        rs += (p0 + p1) + (p2 + p3);
+        pk[c] = pack_bf16(p0, p1);
+        pk[16 + c] = pack_bf16(p2, p3);
+      }
+      l += rs;
+      tmem_st32(tl + s * 64, pk);
+      if (t >= 1 && !wait_warp(&sm.o_done, (t - 1) & 1, wc)) {
+        ok = false;
+        break;
+      }
+      if (__any_sync(0xffffffff, rescale)) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t ov[32];
+          tmem_ld32(tl + 128 + cc * 32, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
+          tmem_st32(tl + 128 + cc * 32, ov);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&sm.p_full[s]);
+    }
+    tmem_wait_st();
+    // agree on the epilogue among the 128 softmax threads
+    named_bar_sync(1, 128);
+    if (threadIdx.x == 0) sm.epi_ok = (n > 0 && !sm.abort_flag) ? 1 : 0;
+    named_bar_sync(1, 128);
+    ok = sm.epi_ok != 0;
+    if (ok) ok = wait_warp(&sm.o_done, (n - 1) & 1, wc);
+    ok = __all_sync(0xffffffff, ok);
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t ov[32];
+        tmem_ld32(tl + 128 + cc * 32, ov);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          pk[c] = pack_bf16(__uint_as_float(ov[2 * c]) * inv_l, __uint_as_float(ov[2 * c + 1]) * inv_l);
+        uint8_t* chunk = sm.q[cc >> 1];
+        const uint32_t u0 = (cc & 1) * 4;
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          *reinterpret_cast<uint4*>(chunk + sw128_offset(r, u0 + e)) =
+              make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+      }
+      const long long row = (long long)i * 128 + r;
+      if (row < N) lse[(long long)bh * N + row] = (m_use + log2f(l)) * 0.69314718055994530942f;
+    }
+    fence_proxy_async_smem();
+    named_bar_sync(1, 128);
+    if (threadIdx.x == 0 && sm.epi_ok) {
+      for (int c = 0; c < CH; ++c) tma_store_3d(&tm_o, sm.q[c], c * 64, i * 128, bh);
+      tma_store_commit();
+      tma_store_wait_all();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+cudaError_t launch_fwd(const FwdArgs& a, int d, cudaStream_t s) {
+  dim3 grid(a.Tm, a.BH);
+  if (d == 128) {
+    const size_t smem = sizeof(FwdSmem<128>) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    fwd_kernel<128><<<grid, 192, smem, s>>>(*a.tm_q, *a.tm_k, *a.tm_v, *a.tm_o, a.row_cnt, a.row_idx, a.lse, a.N,
+                                            a.Tm, a.Tn, a.scale_log2, a.status, a.wait_limit_ns);
+  } else {
+    const size_t smem = sizeof(FwdSmem<64>) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    fwd_kernel<64><<<grid, 192, smem, s>>>(*a.tm_q, *a.tm_k, *a.tm_v, *a.tm_o, a.row_cnt, a.row_idx, a.lse, a.N,
+                                           a.Tm, a.Tn, a.scale_log2, a.status, a.wait_limit_ns);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace spa2

@@ -1,0 +1,72 @@
+// Internal launcher declarations of libspa2 (not part of the C ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace spa2 {
+
+struct MaskOut {
+  int* row_cnt;
+  int* row_idx;
+  float* pbar;       // may be null
+  uint8_t* bitmap;   // may be null
+};
+
+// mask.cu
+cudaError_t launch_pool(const void* q, const void* k, float* qbar, float* kbar, int BH, int N, int d, int Tm, int Tn,
+                        int bq, int bkv, cudaStream_t s);
+cudaError_t launch_pbar_select(const float* qbar, const float* kbar, int BH, int d, int Tm, int Tn, int K,
+                               unsigned long long thr, const MaskOut& out, uint32_t* bits, int W, int* status,
+                               cudaStream_t s);
+size_t pbar_select_max_smem(int d, int Tn);
+cudaError_t launch_select(const float* pbar, int BH, int Tm, int Tn, int K, unsigned long long thr,
+                          const MaskOut& out, uint32_t* bits, int W, int* status, cudaStream_t s);
+cudaError_t launch_csc(const uint32_t* bits, int BH, int Tm, int Tn, int W, int* col_cnt, int* col_idx,
+                       cudaStream_t s);
+
+// attn_fwd.cu
+struct FwdArgs {
+  const CUtensorMap* tm_q;   // box {64, 128, 1}
+  const CUtensorMap* tm_k;   // box {64, 64, 1}
+  const CUtensorMap* tm_v;   // box {64, 64, 1}
+  const CUtensorMap* tm_o;   // box {64, 128, 1}
+  const int* row_cnt;
+  const int* row_idx;
+  float* lse;
+  int BH, N, Tm, Tn;
+  float scale_log2;   // softmax_scale * log2(e)
+  int* status;
+  unsigned long long wait_limit_ns;
+};
+cudaError_t launch_fwd(const FwdArgs& a, int d, cudaStream_t s);
+
+// attn_bwd.cu
+struct BwdArgs {
+  const CUtensorMap* tm_q;    // box {64, 128, 1}
+  const CUtensorMap* tm_k;    // box {64, 64, 1}
+  const CUtensorMap* tm_v;    // box {64, 64, 1}
+  const CUtensorMap* tm_do;   // box {64, 128, 1}
+  const void* o;
+  const void* dout;
+  const float* lse;
+  const int* col_cnt;
+  const int* col_idx;
+  float* dvec;     // [BH, N]
+  float* dq_acc;   // [BH, N, d]
+  void* dq;
+  void* dk;
+  void* dv;
+  int BH, N, Tm, Tn;
+  float scale;        // softmax_scale
+  float scale_log2;   // softmax_scale * log2(e)
+  int* status;
+  unsigned long long wait_limit_ns;
+};
+cudaError_t launch_bwd(const BwdArgs& a, int d, cudaStream_t s);
+
+// api.cu
+cudaError_t launch_timeout_probe(int* status, unsigned long long limit_ns, cudaStream_t s);
+
+}  // namespace spa2
