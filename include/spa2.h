@@ -61,7 +61,8 @@ typedef enum {
   SPA2_ERR_CUDA = 3,           /* a CUDA runtime / driver call failed */
   SPA2_ERR_DEVICE_TIMEOUT = 4, /* a device-side bounded wait ran out */
   SPA2_ERR_WORKSPACE = 5,      /* ws is NULL or smaller than spa2_workspace_bytes */
-  SPA2_ERR_DEVICE_BOUNDS = 6   /* a device-side index check failed (bad mask) */
+  SPA2_ERR_DEVICE_BOUNDS = 6, /* a device-side index check failed (bad mask) */
+  SPA2_ERR_RANGE = 7           /* an input value outside the supported range (|V| > 65504) */
 } spa2_status;
 
 /*
@@ -88,6 +89,9 @@ typedef struct {
 } spa2_mask;
 
 enum { SPA2_OP_MASK = 0, SPA2_OP_FWD = 1, SPA2_OP_BWD = 2, SPA2_OP_SELECT = 3 };
+
+/* Element type of the gradient outputs of spa2_sparse_attn_bwd. */
+enum { SPA2_DTYPE_BF16 = 0, SPA2_DTYPE_F32 = 1 };
 
 /* ABI version of this header (bumped on any incompatible change). */
 #define SPA2_ABI_VERSION 1
@@ -140,16 +144,24 @@ SPA2_API spa2_status spa2_select_blocks(const float* pbar, int B, int H, int Tm,
  * "块稀疏注意力"; gist.science 2C): for every q-block i and every kept kv-block j
  * of row i, S_ij = Q_i K_j^T * softmax_scale, online softmax, O_i += P_ij V_j;
  * masked (i, j) tiles are skipped entirely. No causal mask.
+ * Precision: S = Q K^T takes bf16 operands; P V runs with fp16 operands (P in
+ * [0, 256] and an fp16 copy of V made in the workspace, exact for bf16 V with
+ * |V| <= 65504; larger values are clamped and reported as SPA2_ERR_RANGE),
+ * fp32 accumulation throughout.
  *   q, k, v       : [B, H, N, d] bf16 device pointers (read only)
  *   mask          : host pointer to a spa2_mask; row_cnt/row_idx are read
  *   softmax_scale : logit scale; 0 means 1/sqrt(d)
- *   o             : [B, H, N, d] bf16 device output
+ *   o             : [B, H, N, d] bf16 device output, O rounded to nearest
+ *   o_lo          : optional [B, H, N, d] bf16 device output, the residual
+ *                   bf16(O - o) of the fp32 O (o + o_lo carries ~16 mantissa
+ *                   bits); pass it to the backward for an accurate
+ *                   D = rowsum(dO * O). NULL skips it.
  *   lse           : [B, H, N] fp32 device output (natural-log LSE)
  *   ws            : spa2_workspace_bytes(SPA2_OP_FWD, ...) bytes
  */
-SPA2_API spa2_status spa2_sparse_attn_fwd(const void* q, const void* k, const void* v, int B, int H, int N, int d, int bq,
-                                 int bkv, const spa2_mask* mask, float softmax_scale, void* o, float* lse, void* ws,
-                                 size_t ws_bytes, spa2_stream_t stream);
+SPA2_API spa2_status spa2_sparse_attn_fwd(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                                          int bq, int bkv, const spa2_mask* mask, float softmax_scale, void* o,
+                                          void* o_lo, float* lse, void* ws, size_t ws_bytes, spa2_stream_t stream);
 
 /*
  * Step 4 backward through the same block mask (the trainable part;
@@ -158,18 +170,25 @@ SPA2_API spa2_status spa2_sparse_attn_fwd(const void* q, const void* k, const vo
  *   dS_ij = P_ij * (dP_ij - D_i),  dQ_i = sum_j dS_ij K_j * scale,
  *   dK_j = sum_i dS_ij^T Q_i * scale.
  * The mask is held constant (no gradient through pooling or selection).
- *   q, k, v, o, dout : [B, H, N, d] bf16 device pointers (read only); o and
- *                      lse are the forward outputs for the same mask
+ * Precision: P and dS enter the dV, dK and dQ tensor-core products as
+ * hi + lo bf16 pairs (about 16 mantissa bits) with fp32 accumulation, and D
+ * uses o + o_lo when o_lo is given, so the gradients carry fp32-level error
+ * before their final store.
+ *   q, k, v, o, dout : [B, H, N, d] bf16 device pointers (read only); o, o_lo
+ *                      and lse are the forward outputs for the same mask
+ *   o_lo             : optional [B, H, N, d] bf16 residual of O (or NULL)
  *   lse              : [B, H, N] fp32 device pointer
  *   mask             : host pointer to a spa2_mask; col_cnt/col_idx are read
- *   dq, dk, dv       : [B, H, N, d] bf16 device outputs
- *   ws               : spa2_workspace_bytes(SPA2_OP_BWD, ...) bytes (holds the
- *                      fp32 dQ accumulator and D)
+ *   dq, dk, dv       : [B, H, N, d] device outputs of type grad_dtype
+ *   grad_dtype       : SPA2_DTYPE_BF16 or SPA2_DTYPE_F32
+ *   ws               : spa2_workspace_bytes(SPA2_OP_BWD, ...) bytes (holds D
+ *                      and, for bf16 gradients, the fp32 dQ accumulator)
  */
-SPA2_API spa2_status spa2_sparse_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
-                                 const void* dout, int B, int H, int N, int d, int bq, int bkv, const spa2_mask* mask,
-                                 float softmax_scale, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
-                                 spa2_stream_t stream);
+SPA2_API spa2_status spa2_sparse_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                                          const void* o_lo, const float* lse, const void* dout, int B, int H, int N,
+                                          int d, int bq, int bkv, const spa2_mask* mask, float softmax_scale,
+                                          void* dq, void* dk, void* dv, int grad_dtype, void* ws, size_t ws_bytes,
+                                          spa2_stream_t stream);
 
 /*
  * Synchronises `stream`, then reads and clears the status word at the start

@@ -24,6 +24,44 @@ def assert_close(actual, expected, what, max_abs=MAX_ABS, rel_l1=REL_L1):
     return ma, rl1
 
 
+def bf16_half_ulp(x):
+    """Half a bf16 ulp of |x| (the rounding error of storing x as bf16)."""
+    a = np.maximum(np.abs(np.asarray(x, dtype=np.float64)), 2.0 ** -126)
+    return np.exp2(np.floor(np.log2(a)) - 8)
+
+
+def assert_close_bf16_out(actual, expected, what, max_abs=MAX_ABS, rel_l1=REL_L1):
+    """bf16 outputs: the stated tolerance plus half a bf16 ulp of each expected value."""
+    a = np.asarray(actual, dtype=np.float64)
+    e = np.asarray(expected, dtype=np.float64)
+    assert a.shape == e.shape, (what, a.shape, e.shape)
+    err = np.abs(a - e)
+    excess = err - (max_abs + bf16_half_ulp(e))
+    rl1 = float(err.sum() / max(np.abs(e).sum(), 1e-300))
+    assert excess.max() <= 0 and rl1 <= rel_l1, f"{what}: worst excess {excess.max():.3e} rel_l1={rl1:.3e}"
+
+
+class Accum:
+    """Max-abs per element and relative L1 over several sampled blocks of one tensor."""
+
+    def __init__(self, what):
+        self.what, self.err, self.ref, self.ma = what, 0.0, 0.0, 0.0
+
+    def add(self, actual, expected):
+        a = np.asarray(actual, dtype=np.float64)
+        e = np.asarray(expected, dtype=np.float64)
+        assert a.shape == e.shape and np.isfinite(a).all()
+        d = np.abs(a - e)
+        self.ma = max(self.ma, float(d.max()))
+        self.err += float(d.sum())
+        self.ref += float(np.abs(e).sum())
+
+    def check(self, max_abs=MAX_ABS, rel_l1=REL_L1):
+        rl1 = self.err / max(self.ref, 1e-300)
+        assert self.ma <= max_abs and rl1 <= rel_l1, f"{self.what}: max_abs={self.ma:.3e} rel_l1={rl1:.3e}"
+        return self.ma, rl1
+
+
 def csr_to_dense(row_cnt, row_idx, Tn):
     """bool [.., Tm, Tn] from CSR numpy arrays; checks ids ascending and in range."""
     cnt = np.asarray(row_cnt)

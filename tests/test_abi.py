@@ -28,7 +28,7 @@ def test_exports_every_header_symbol(L):
 
 def test_version_and_status_strings(L):
     assert b.spa2_abi_version() == 1
-    for code in range(7):
+    for code in range(8):
         assert b.status_string(code)
     assert b.status_string(99) == "unknown status"
 
@@ -38,7 +38,7 @@ def test_workspace_sizes(L):
     Tm, Tn = 256, 512
     m = b.spa2_workspace_bytes(b.OP_MASK, B, H, N, d)
     assert m >= 256 + B * H * (Tm + Tn) * d * 4 + B * H * Tm * 16 * 4
-    assert b.spa2_workspace_bytes(b.OP_FWD, B, H, N, d) == 256
+    assert b.spa2_workspace_bytes(b.OP_FWD, B, H, N, d) == 256 + B * H * N * d * 2   # status + fp16 V
     assert b.spa2_workspace_bytes(b.OP_BWD, B, H, N, d) >= 256 + B * H * N * (d + 1) * 4
     assert b.spa2_workspace_bytes(b.OP_SELECT, 2, 3, 5, 40, 0, 0) == 256 + 256   # 2*3*5*2 words = 240 B
     # unsupported shapes report 0
@@ -72,17 +72,21 @@ def test_argument_errors_are_synchronous(L):
     assert b.spa2_block_mask(fake, fake, 1, 1, 128, 128, 128, 64, 0.1, 0.5, m2, fake, 1 << 30,
                              None) == b.ERR_INVALID_ARG
     # forward / backward
-    assert b.spa2_sparse_attn_fwd(fake, fake, fake, 1, 1, 128, 128, 128, 64, m, 0.0, fake, None, fake, 256,
-                                  None) == b.ERR_INVALID_ARG
-    assert b.spa2_sparse_attn_fwd(fake, fake, fake, 1, 1, 128, 128, 128, 64, m, -1.0, fake, fake, fake, 256,
+    assert b.spa2_sparse_attn_fwd(fake, fake, fake, 1, 1, 128, 128, 128, 64, m, 0.0, fake, None, None, fake, 256,
+                                  None) == b.ERR_INVALID_ARG                        # no lse
+    assert b.spa2_sparse_attn_fwd(fake, fake, fake, 1, 1, 128, 128, 128, 64, m, 0.0, fake, fake + 8, fake, fake,
+                                  256, None) == b.ERR_INVALID_ARG                   # misaligned o_lo
+    assert b.spa2_sparse_attn_fwd(fake, fake, fake, 1, 1, 128, 128, 128, 64, m, -1.0, fake, None, fake, fake, 256,
                                   None) == b.ERR_UNSUPPORTED
-    assert b.spa2_sparse_attn_fwd(fake, fake, fake, 1, 1, 128, 128, 128, 64, m, 0.0, fake, fake, fake, 255,
+    assert b.spa2_sparse_attn_fwd(fake, fake, fake, 1, 1, 128, 128, 128, 64, m, 0.0, fake, None, fake, fake, 255,
                                   None) == b.ERR_WORKSPACE
-    assert b.spa2_sparse_attn_bwd(fake, fake, fake, fake, fake, fake, 1, 1, 128, 128, 128, 64, m, 0.0, fake, fake,
-                                  fake, fake, 1 << 30, None) == b.ERR_INVALID_ARG   # mask has no CSC
+    assert b.spa2_sparse_attn_bwd(fake, fake, fake, fake, None, fake, fake, 1, 1, 128, 128, 128, 64, m, 0.0, fake,
+                                  fake, fake, b.DTYPE_F32, fake, 1 << 30, None) == b.ERR_INVALID_ARG  # no CSC
     mc = b.spa2_mask(fake, fake, fake, fake, None, None)
-    assert b.spa2_sparse_attn_bwd(fake, fake, fake, fake, fake, fake, 1, 1, 128, 128, 128, 64, mc, 0.0, fake, fake,
-                                  fake, fake, 1000, None) == b.ERR_WORKSPACE
+    assert b.spa2_sparse_attn_bwd(fake, fake, fake, fake, None, fake, fake, 1, 1, 128, 128, 128, 64, mc, 0.0, fake,
+                                  fake, fake, b.DTYPE_F32, fake, 1000, None) == b.ERR_WORKSPACE
+    assert b.spa2_sparse_attn_bwd(fake, fake, fake, fake, None, fake, fake, 1, 1, 128, 128, 128, 64, mc, 0.0, fake,
+                                  fake, fake, 7, fake, 1 << 30, None) == b.ERR_UNSUPPORTED      # bad grad dtype
     assert b.spa2_select_blocks(fake, 1, 1, 4, 5000, 0.1, 0.5, m, fake, 1 << 30, None) == b.ERR_UNSUPPORTED
     assert b.spa2_debug_timeout_probe(None, 0, None) == b.ERR_WORKSPACE
     assert b.spa2_debug_set_wait_limit_ns(0) == b.OK

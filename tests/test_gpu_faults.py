@@ -74,3 +74,17 @@ def test_bad_column_count_is_reported_by_backward():
         s.check(b.OP_BWD)
     assert e.value.code == b.ERR_DEVICE_BOUNDS
     _small_pass()
+
+
+def test_v_outside_fp16_range_is_reported():
+    q, k, v = synth.gaussian_with_sinks(B=1, H=1, N=256, d=128, seed=5, device="cuda")
+    v = v.clone()
+    v[0, 0, 17, 3] = 1e6
+    s = b.Spa2(1, 1, 256, 128)
+    m = s.block_mask(q, k, 0.5, 0.5)
+    o, _ = s.fwd(q, k, v, m)
+    with pytest.raises(b.Spa2Error) as e:
+        s.check(b.OP_FWD)
+    assert e.value.code == b.ERR_RANGE
+    assert torch.isfinite(o.float()).all()      # clamped, never inf
+    _small_pass()

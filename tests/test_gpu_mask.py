@@ -92,7 +92,7 @@ def _hard_rows(rng, Tn, nrows):
             x = rng.dirichlet(np.full(Tn, 1.0))
             x[rng.integers(0, Tn, Tn // 3)] = x[0]
         elif kind == 3:                         # sink + near-uniform tail
-            x = np.full(Tn, 0.4 / (Tn - 1)); x[rng.integers(Tn)] = 0.6
+            x = np.full(Tn, 0.4 / max(Tn - 1, 1)); x[rng.integers(Tn)] = 0.6
         elif kind == 4:                         # one-hot (Top-p reaches p with one block)
             x = np.zeros(Tn); x[rng.integers(Tn)] = 1.0
         else:                                   # tiny values below 2^-32 mixed in

@@ -20,8 +20,10 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libspa2.so")
 HEADER = os.path.join(os.path.dirname(HERE), "include", "spa2.h")
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_DEVICE_TIMEOUT, ERR_WORKSPACE, ERR_DEVICE_BOUNDS = range(7)
+(OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_DEVICE_TIMEOUT, ERR_WORKSPACE, ERR_DEVICE_BOUNDS,
+ ERR_RANGE) = range(8)
 OP_MASK, OP_FWD, OP_BWD, OP_SELECT = range(4)
+DTYPE_BF16, DTYPE_F32 = 0, 1
 BQ, BKV = 128, 64
 
 
@@ -56,10 +58,10 @@ _SIGS = {
                               ctypes.c_size_t, ctypes.c_void_p]),
     "spa2_sparse_attn_fwd": (ctypes.c_int, [ctypes.c_void_p] * 3 + [ctypes.c_int] * 6
                              + [ctypes.POINTER(spa2_mask), ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
-                                ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
-    "spa2_sparse_attn_bwd": (ctypes.c_int, [ctypes.c_void_p] * 6 + [ctypes.c_int] * 6
-                             + [ctypes.POINTER(spa2_mask), ctypes.c_float] + [ctypes.c_void_p] * 4
-                             + [ctypes.c_size_t, ctypes.c_void_p]),
+                                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "spa2_sparse_attn_bwd": (ctypes.c_int, [ctypes.c_void_p] * 7 + [ctypes.c_int] * 6
+                             + [ctypes.POINTER(spa2_mask), ctypes.c_float] + [ctypes.c_void_p] * 3
+                             + [ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "spa2_stream_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
     "spa2_debug_set_wait_limit_ns": (ctypes.c_int, [ctypes.c_longlong]),
     "spa2_debug_timeout_probe": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
@@ -116,15 +118,16 @@ def spa2_select_blocks(pbar, B, H, Tm, Tn, k_frac, p_frac, mask: spa2_mask, ws, 
     return lib().spa2_select_blocks(pbar, B, H, Tm, Tn, k_frac, p_frac, ctypes.byref(mask), ws, ws_bytes, stream)
 
 
-def spa2_sparse_attn_fwd(q, k, v, B, H, N, d, bq, bkv, mask: spa2_mask, scale, o, lse, ws, ws_bytes, stream) -> int:
-    return lib().spa2_sparse_attn_fwd(q, k, v, B, H, N, d, bq, bkv, ctypes.byref(mask), scale, o, lse, ws, ws_bytes,
-                                      stream)
+def spa2_sparse_attn_fwd(q, k, v, B, H, N, d, bq, bkv, mask: spa2_mask, scale, o, o_lo, lse, ws, ws_bytes,
+                         stream) -> int:
+    return lib().spa2_sparse_attn_fwd(q, k, v, B, H, N, d, bq, bkv, ctypes.byref(mask), scale, o, o_lo, lse, ws,
+                                      ws_bytes, stream)
 
 
-def spa2_sparse_attn_bwd(q, k, v, o, lse, dout, B, H, N, d, bq, bkv, mask: spa2_mask, scale, dq, dk, dv, ws,
-                         ws_bytes, stream) -> int:
-    return lib().spa2_sparse_attn_bwd(q, k, v, o, lse, dout, B, H, N, d, bq, bkv, ctypes.byref(mask), scale, dq, dk,
-                                      dv, ws, ws_bytes, stream)
+def spa2_sparse_attn_bwd(q, k, v, o, o_lo, lse, dout, B, H, N, d, bq, bkv, mask: spa2_mask, scale, dq, dk, dv,
+                         grad_dtype, ws, ws_bytes, stream) -> int:
+    return lib().spa2_sparse_attn_bwd(q, k, v, o, o_lo, lse, dout, B, H, N, d, bq, bkv, ctypes.byref(mask), scale,
+                                      dq, dk, dv, grad_dtype, ws, ws_bytes, stream)
 
 
 def spa2_stream_status(ws, stream) -> int:
@@ -184,7 +187,8 @@ class Spa2:
         self.ws_bytes = {op: L.spa2_workspace_bytes(op, B, H, N, d, BQ, BKV) for op in (OP_MASK, OP_FWD, OP_BWD)}
         if min(self.ws_bytes.values()) == 0:
             raise Spa2Error(ERR_UNSUPPORTED, f"shape B={B} H={H} N={N} d={d}")
-        self.ws = {op: torch.empty(n, dtype=torch.uint8, device=device) for op, n in self.ws_bytes.items()}
+        # zero-filled so that the status word of an op never run reads as OK
+        self.ws = {op: torch.zeros(n, dtype=torch.uint8, device=device) for op, n in self.ws_bytes.items()}
         self.with_pbar, self.with_bitmap = with_pbar, with_bitmap
 
     def new_mask(self) -> Mask:
@@ -203,27 +207,37 @@ class Spa2:
                                float(p_frac), cm, ws.data_ptr(), ws.numel(), _stream(self.torch)), "spa2_block_mask")
         return mask
 
-    def fwd(self, q, k, v, mask: Mask, scale=0.0, o=None, lse=None):
+    def fwd(self, q, k, v, mask: Mask, scale=0.0, o=None, lse=None, o_lo=None, want_o_lo=True):
+        """O (bf16), LSE (fp32) and, if wanted, O's bf16 residual for the backward."""
         t = self.torch
         o = t.empty_like(q) if o is None else o
+        if want_o_lo and o_lo is None:
+            o_lo = t.empty_like(q)
         lse = t.empty(self.B, self.H, self.N, dtype=t.float32, device=q.device) if lse is None else lse
         cm = mask.c()
         ws = self.ws[OP_FWD]
         _check(spa2_sparse_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), self.B, self.H, self.N, self.d, BQ,
-                                    BKV, cm, float(scale), o.data_ptr(), lse.data_ptr(), ws.data_ptr(), ws.numel(),
-                                    _stream(t)), "spa2_sparse_attn_fwd")
+                                    BKV, cm, float(scale), o.data_ptr(), None if o_lo is None else o_lo.data_ptr(),
+                                    lse.data_ptr(), ws.data_ptr(), ws.numel(), _stream(t)), "spa2_sparse_attn_fwd")
+        self.o_lo = o_lo
         return o, lse
 
-    def bwd(self, q, k, v, o, lse, dout, mask: Mask, scale=0.0, dq=None, dk=None, dv=None):
+    def bwd(self, q, k, v, o, lse, dout, mask: Mask, scale=0.0, dq=None, dk=None, dv=None, o_lo="auto",
+            grad_dtype=DTYPE_F32):
+        """dQ, dK, dV (fp32 by default; grad_dtype=DTYPE_BF16 for bf16)."""
         t = self.torch
-        dq = t.empty_like(q) if dq is None else dq
-        dk = t.empty_like(k) if dk is None else dk
-        dv = t.empty_like(v) if dv is None else dv
+        gt = t.float32 if grad_dtype == DTYPE_F32 else t.bfloat16
+        dq = t.empty(q.shape, dtype=gt, device=q.device) if dq is None else dq
+        dk = t.empty(k.shape, dtype=gt, device=q.device) if dk is None else dk
+        dv = t.empty(v.shape, dtype=gt, device=q.device) if dv is None else dv
+        if isinstance(o_lo, str):
+            o_lo = getattr(self, "o_lo", None)
         cm = mask.c()
         ws = self.ws[OP_BWD]
-        _check(spa2_sparse_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                                    dout.data_ptr(), self.B, self.H, self.N, self.d, BQ, BKV, cm, float(scale),
-                                    dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws.numel(),
+        _check(spa2_sparse_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                    None if o_lo is None else o_lo.data_ptr(), lse.data_ptr(), dout.data_ptr(),
+                                    self.B, self.H, self.N, self.d, BQ, BKV, cm, float(scale), dq.data_ptr(),
+                                    dk.data_ptr(), dv.data_ptr(), int(grad_dtype), ws.data_ptr(), ws.numel(),
                                     _stream(t)), "spa2_sparse_attn_bwd")
         return dq, dk, dv
 

@@ -105,14 +105,14 @@ static EncodeTiledFn encode_fn() {
 
 // [BH, N, d] bf16 viewed as a 3-D tensor {d, N, BH}; box {64, rows, 1}, 128-byte
 // swizzle; rows past N of a head read as zero (no spill into the next head).
-static bool make_map(CUtensorMap* m, const void* ptr, const Shape& s, int rows) {
+static bool make_map(CUtensorMap* m, const void* ptr, const Shape& s, int rows, bool f16 = false) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {(cuuint64_t)s.d, (cuuint64_t)s.N, (cuuint64_t)s.BH};
   cuuint64_t strides[2] = {(cuuint64_t)s.d * 2, (cuuint64_t)s.N * s.d * 2};
   cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+  CUresult r = fn(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -170,6 +170,7 @@ const char* spa2_status_string(spa2_status s) {
     case SPA2_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
     case SPA2_ERR_WORKSPACE: return "workspace missing or too small";
     case SPA2_ERR_DEVICE_BOUNDS: return "device-side index check failed";
+    case SPA2_ERR_RANGE: return "input value outside the supported range";
   }
   return "unknown status";
 }
@@ -186,7 +187,7 @@ size_t spa2_workspace_bytes(int op, int B, int H, int N, int d, int bq, int bkv)
   if (!shape_ok(B, H, N, d, bq, bkv, &s, &err)) return 0;
   switch (op) {
     case SPA2_OP_MASK: return mask_ws(nullptr, s).bytes;
-    case SPA2_OP_FWD: return 256;
+    case SPA2_OP_FWD: return 256 + al256((size_t)s.BH * s.N * s.d * 2);  // status + fp16 V
     case SPA2_OP_BWD: return bwd_ws(nullptr, s).bytes;
   }
   return 0;
@@ -239,41 +240,46 @@ spa2_status spa2_select_blocks(const float* pbar, int B, int H, int Tm, int Tn, 
 }
 
 spa2_status spa2_sparse_attn_fwd(const void* q, const void* k, const void* v, int B, int H, int N, int d, int bq,
-                                 int bkv, const spa2_mask* mask, float softmax_scale, void* o, float* lse, void* ws,
-                                 size_t ws_bytes, spa2_stream_t stream) {
+                                 int bkv, const spa2_mask* mask, float softmax_scale, void* o, void* o_lo, float* lse,
+                                 void* ws, size_t ws_bytes, spa2_stream_t stream) {
   Shape s;
   spa2_status err;
   if (!q || !k || !v || !o || !lse || !mask || !mask->row_cnt || !mask->row_idx) return SPA2_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(o_lo, 16) ||
+      !aligned(lse, 4))
     return SPA2_ERR_INVALID_ARG;
   if (!shape_ok(B, H, N, d, bq, bkv, &s, &err)) return err;
   if (!(softmax_scale >= 0.f) || isinf(softmax_scale)) return SPA2_ERR_UNSUPPORTED;
   if (!ws || !aligned(ws, 256)) return SPA2_ERR_WORKSPACE;
-  if (ws_bytes < 256) return SPA2_ERR_WORKSPACE;
+  if (ws_bytes < 256 + al256((size_t)s.BH * s.N * s.d * 2)) return SPA2_ERR_WORKSPACE;
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)d);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  CUtensorMap tq, tk, tv, to;
-  if (!make_map(&tq, q, s, 128) || !make_map(&tk, k, s, 64) || !make_map(&tv, v, s, 64) || !make_map(&to, o, s, 128))
+  void* v16 = static_cast<char*>(ws) + 256;
+  CUtensorMap tq, tk, tv, to, tolo;
+  if (!make_map(&tq, q, s, 128) || !make_map(&tk, k, s, 64) || !make_map(&tv, v16, s, 64, true) ||
+      !make_map(&to, o, s, 128) || !make_map(&tolo, o_lo ? o_lo : o, s, 128))
     return SPA2_ERR_CUDA;
   int* status = static_cast<int*>(ws);
   SPA2_CUDA_TRY(cudaMemsetAsync(status, 0, 4, st));
-  FwdArgs a{&tq, &tk, &tv, &to, mask->row_cnt, mask->row_idx, lse, (int)s.BH, s.N, s.Tm, s.Tn,
-            scale * 1.4426950408889634f, status, g_wait_limit_ns};
+  SPA2_CUDA_TRY(launch_v_to_f16(v, v16, s.BH * s.N * s.d, status, st));
+  FwdArgs a{&tq, &tk, &tv, &to, &tolo, o_lo != nullptr, mask->row_cnt, mask->row_idx, lse, (int)s.BH, s.N, s.Tm,
+            s.Tn, scale * 1.4426950408889634f, status, g_wait_limit_ns};
   SPA2_CUDA_TRY(launch_fwd(a, d, st));
   return SPA2_OK;
 }
 
-spa2_status spa2_sparse_attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
-                                 const void* dout, int B, int H, int N, int d, int bq, int bkv, const spa2_mask* mask,
-                                 float softmax_scale, void* dq, void* dk, void* dv, void* ws, size_t ws_bytes,
-                                 spa2_stream_t stream) {
+spa2_status spa2_sparse_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* o_lo,
+                                 const float* lse, const void* dout, int B, int H, int N, int d, int bq, int bkv,
+                                 const spa2_mask* mask, float softmax_scale, void* dq, void* dk, void* dv,
+                                 int grad_dtype, void* ws, size_t ws_bytes, spa2_stream_t stream) {
   Shape s;
   spa2_status err;
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !mask || !mask->col_cnt || !mask->col_idx)
     return SPA2_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||
-      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4))
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(o_lo, 16) ||
+      !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4))
     return SPA2_ERR_INVALID_ARG;
+  if (grad_dtype != SPA2_DTYPE_BF16 && grad_dtype != SPA2_DTYPE_F32) return SPA2_ERR_UNSUPPORTED;
   if (!shape_ok(B, H, N, d, bq, bkv, &s, &err)) return err;
   if (!(softmax_scale >= 0.f) || isinf(softmax_scale)) return SPA2_ERR_UNSUPPORTED;
   if (!ws || !aligned(ws, 256)) return SPA2_ERR_WORKSPACE;
@@ -286,8 +292,9 @@ spa2_status spa2_sparse_attn_bwd(const void* q, const void* k, const void* v, co
       !make_map(&tdo, dout, s, 128))
     return SPA2_ERR_CUDA;
   SPA2_CUDA_TRY(cudaMemsetAsync(w.status, 0, 4, st));
-  BwdArgs a{&tq, &tk, &tv, &tdo, o, dout, lse, mask->col_cnt, mask->col_idx, w.dvec, w.dq_acc, dq, dk, dv,
-            (int)s.BH, s.N, s.Tm, s.Tn, scale, scale * 1.4426950408889634f, w.status, g_wait_limit_ns};
+  BwdArgs a{&tq, &tk, &tv, &tdo, o, o_lo, dout, lse, mask->col_cnt, mask->col_idx, w.dvec, w.dq_acc, dq, dk, dv,
+            grad_dtype == SPA2_DTYPE_F32 ? 1 : 0, (int)s.BH, s.N, s.Tm, s.Tn, scale, scale * 1.4426950408889634f,
+            w.status, g_wait_limit_ns};
   SPA2_CUDA_TRY(launch_bwd(a, d, st));
   return SPA2_OK;
 }

@@ -5,7 +5,7 @@
 //   dV_j += P^T dO_i      dP = dO_i V_j^T      dS = P * (dP - D_i)
 //   dQ_i += dS K_j * sc   dK_j += dS^T Q_i * sc,  D_i = rowsum(dO_i * O_i).
 //
-// bwd_pre_kernel   D = rowsum(dO * O) (fp32) and zeroes the fp32 dQ accumulator.
+// bwd_pre_kernel   D = rowsum(dO * (O + O_lo)) in fp32 and zeroes the fp32 dQ.
 // bwd_kernel       one CTA per (kv-block j, head), looping over the q-blocks i
 //                  that keep j (CSC column of j). Every GEMM is an M=128 tcgen05
 //                  MMA with fp32 accumulation in TMEM:
@@ -15,14 +15,17 @@
 //                    dK^T += Q_i^T dS  M=d       N=64 (kv) K=128  A,B MN-major
 //                    dQ  = dS K_j      M=128 (q) N=d       K=64   A K-, B MN-major
 //                  Warps 0-3 turn S, dP into P, dS (thread = query row) and write
-//                  them as bf16 into 128-byte-swizzled smem tiles that serve as
-//                  both the K-major A operand of dQ and the MN-major B operand of
-//                  dV^T / dK^T. Warps 4-7 drain each dQ tile from TMEM into the
-//                  fp32 accumulator with 16-byte vector atomics. Warp 8 is the
-//                  TMA producer, warp 9 issues the MMAs and owns TMEM.
-//                  For d = 64 the dV^T / dK^T MMAs still run at M = 128 (the
-//                  upper 64 lanes repeat the lower ones and are ignored).
-// dq_convert_kernel  fp32 dQ accumulator -> bf16 dQ.
+//                  each as a hi + lo pair of bf16 tiles (x = hi + lo to about 16
+//                  mantissa bits) into 128-byte-swizzled smem; the tiles serve
+//                  as the K-major A operand of dQ and the MN-major B operand of
+//                  dV^T / dK^T, and each of those products runs once per half,
+//                  so P and dS reach the fp32 accumulators with fp32-level error.
+//                  Warps 4-7 drain each dQ tile from TMEM into the fp32 dQ (the
+//                  output itself for fp32 gradients) with 16-byte vector
+//                  atomics. Warp 8 is the TMA producer; warp 9 issues the MMAs
+//                  and owns TMEM. For d = 64 the dV^T / dK^T MMAs still run at
+//                  M = 128 (the upper 64 lanes repeat the lower ones, ignored).
+// dq_convert_kernel  fp32 dQ -> bf16 dQ (bf16 gradients only).
 //
 // TMEM columns: S[2] 0..127, dP[2] 128..255, dV^T 256..319, dK^T 320..383,
 // dQ 384..384+d.
@@ -42,8 +45,8 @@ struct BwdSmem {
   alignas(1024) uint8_t v[CH][64 * 128];
   alignas(1024) uint8_t q[2][CH][128 * 128];
   alignas(1024) uint8_t dO[2][CH][128 * 128];
-  alignas(1024) uint8_t p[128 * 128];    // P  [128 q][64 kv] bf16, swizzled rows
-  alignas(1024) uint8_t ds[128 * 128];   // dS [128 q][64 kv] bf16, swizzled rows
+  alignas(1024) uint8_t p[2][128 * 128];   // P  [128 q][64 kv]: hi, lo bf16 tiles
+  alignas(1024) uint8_t ds[2][128 * 128];  // dS [128 q][64 kv]: hi, lo bf16 tiles
   uint64_t kv_full;
   uint64_t qd_full[2], qd_empty[2], sdp_full[2];
   uint64_t pds_full, pds_empty, dq_full, dq_empty, acc_done, drain;
@@ -57,6 +60,12 @@ SPA2_DEV bool wait_warp(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
   return __all_sync(0xffffffff, ok);
 }
 
+SPA2_DEV void split_bf16(float a, float b, uint32_t& hi, uint32_t& lo) {
+  hi = pack_bf16(a, b);
+  const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hi));
+  lo = pack_bf16(a - f.x, b - f.y);
+}
+
 }  // namespace
 
 template <int D>
@@ -66,8 +75,8 @@ __global__ void __launch_bounds__(320, 1) bwd_kernel(const __grid_constant__ CUt
                                                      const __grid_constant__ CUtensorMap tm_do,
                                                      const float* __restrict__ lse, const float* __restrict__ dvec,
                                                      const int* __restrict__ col_cnt, const int* __restrict__ col_idx,
-                                                     float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dk,
-                                                     __nv_bfloat16* __restrict__ dv, int N, int Tm, int Tn,
+                                                     float* __restrict__ dq32, void* __restrict__ dk,
+                                                     void* __restrict__ dv, int grad_f32, int N, int Tm, int Tn,
                                                      float scale, float scale_log2, int* status,
                                                      unsigned long long wait_limit_ns) {
   constexpr int CH = D / 64;
@@ -76,6 +85,7 @@ __global__ void __launch_bounds__(320, 1) bwd_kernel(const __grid_constant__ CUt
   constexpr uint32_t IDESC_Q = idesc_bf16_f32(128, D, false, true);
   constexpr uint32_t QT_BYTES = 128 * D * 2;
   constexpr uint32_t KV_BYTES = 64 * D * 2;
+  constexpr uint32_t HALF = 128 * 128;  // bytes from a hi tile to its lo tile
   // MN-major A operand (dO^T, Q^T): stride between the two 64-row halves of M = d
   constexpr uint32_t LBO_DT = (D == 128) ? 128 * 128 : 0;
   constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 320, T_DQ = 384;
@@ -161,10 +171,9 @@ __global__ void __launch_bounds__(320, 1) bwd_kernel(const __grid_constant__ CUt
   } else if (warp == 9) {
     // ---------------- MMA issuer ----------------
     if (lane == 0 && n > 0) {
-      const uint32_t p_addr = smem_u32(sm.p), ds_addr = smem_u32(sm.ds);
+      const uint32_t p_addr = smem_u32(sm.p[0]), ds_addr = smem_u32(sm.ds[0]);
       if (wait_bar(&sm.kv_full, 0, wc)) {
-        bool ok = true;
-        for (int t = 0; t <= n && ok; ++t) {
+        for (int t = 0; t <= n; ++t) {
           if (t < n) {
             const int s = t & 1;
             if (!wait_bar(&sm.qd_full[s], (t >> 1) & 1, wc)) break;
@@ -187,24 +196,33 @@ __global__ void __launch_bounds__(320, 1) bwd_kernel(const __grid_constant__ CUt
             const int u = t - 1, su = u & 1;
             if (!wait_bar(&sm.pds_full, u & 1, wc)) break;
             tc_fence_after();
-            // dV^T += dO^T P and dK^T += Q^T dS, K = 128 query rows
+            // dV^T += dO^T (P_hi + P_lo); dK^T += Q^T (dS_hi + dS_lo); K = 128 query rows
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              mma_ss(tmem + T_DV, sdesc_sw128(smem_u32(sm.dO[su][0]) + kk * 2048, LBO_DT, 1024),
-                     sdesc_sw128(p_addr + kk * 2048, 0, 1024), IDESC_T, (u > 0 || kk > 0) ? 1u : 0u);
+            for (int part = 0; part < 2; ++part) {
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk)
+                mma_ss(tmem + T_DV, sdesc_sw128(smem_u32(sm.dO[su][0]) + kk * 2048, LBO_DT, 1024),
+                       sdesc_sw128(p_addr + part * HALF + kk * 2048, 0, 1024), IDESC_T,
+                       (u > 0 || part > 0 || kk > 0) ? 1u : 0u);
             }
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              mma_ss(tmem + T_DK, sdesc_sw128(smem_u32(sm.q[su][0]) + kk * 2048, LBO_DT, 1024),
-                     sdesc_sw128(ds_addr + kk * 2048, 0, 1024), IDESC_T, (u > 0 || kk > 0) ? 1u : 0u);
+            for (int part = 0; part < 2; ++part) {
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk)
+                mma_ss(tmem + T_DK, sdesc_sw128(smem_u32(sm.q[su][0]) + kk * 2048, LBO_DT, 1024),
+                       sdesc_sw128(ds_addr + part * HALF + kk * 2048, 0, 1024), IDESC_T,
+                       (u > 0 || part > 0 || kk > 0) ? 1u : 0u);
             }
-            // dQ tile = dS K_j, K = 64 kv rows; TMEM dQ must have been drained
+            // dQ tile = (dS_hi + dS_lo) K_j, K = 64 kv rows; TMEM dQ must have been drained
             if (u >= 1 && !wait_bar(&sm.dq_empty, (u - 1) & 1, wc)) break;
             tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              mma_ss(tmem + T_DQ, sdesc_sw128(ds_addr + kk * 32, 16, 1024),
-                     sdesc_sw128(smem_u32(sm.k[0]) + kk * 2048, 64 * 128, 1024), IDESC_Q, kk > 0 ? 1u : 0u);
+            for (int part = 0; part < 2; ++part) {
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                mma_ss(tmem + T_DQ, sdesc_sw128(ds_addr + part * HALF + kk * 32, 16, 1024),
+                       sdesc_sw128(smem_u32(sm.k[0]) + kk * 2048, 64 * 128, 1024), IDESC_Q,
+                       (part > 0 || kk > 0) ? 1u : 0u);
             }
             mma_commit(&sm.dq_full);
             mma_commit(&sm.qd_empty[su]);
@@ -224,7 +242,7 @@ __global__ void __launch_bounds__(320, 1) bwd_kernel(const __grid_constant__ CUt
       if (!wait_warp(&sm.dq_full, t & 1, wc)) break;
       tc_fence_after();
       const long long row = (long long)q_list[t] * 128 + r;
-      float4* dst = reinterpret_cast<float4*>(dq_acc + ((long long)bh * N + row) * D);
+      float4* dst = reinterpret_cast<float4*>(dq32 + ((long long)bh * N + row) * D);
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t v[32];
@@ -258,7 +276,11 @@ __global__ void __launch_bounds__(320, 1) bwd_kernel(const __grid_constant__ CUt
       const bool rvalid = row < N;
       const float lse2 = rvalid ? lse[(long long)bh * N + row] * LOG2E : INFINITY;
       const float Dr = rvalid ? dvec[(long long)bh * N + row] : 0.f;
-      uint32_t pk[32], dk_[32];
+      // the P / dS tiles of the previous tile must have been consumed
+      if (t >= 1 && !wait_warp(&sm.pds_empty, (t - 1) & 1, wc)) {
+        ok = false;
+        break;
+      }
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t sa[32], pa[32];
@@ -266,39 +288,42 @@ __global__ void __launch_bounds__(320, 1) bwd_kernel(const __grid_constant__ CUt
         tmem_ld32(tl + T_DP + s * 64 + h * 32, pa);
         tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          float p0 = fast_exp2(fmaf(__uint_as_float(sa[c]), scale_log2, -lse2));
-          float p1 = fast_exp2(fmaf(__uint_as_float(sa[c + 1]), scale_log2, -lse2));
-          if (h * 32 + c >= kv_valid) p0 = 0.f;
-          if (h * 32 + c + 1 >= kv_valid) p1 = 0.f;
-          pk[h * 16 + c / 2] = pack_bf16(p0, p1);
-          dk_[h * 16 + c / 2] =
-              pack_bf16(p0 * (__uint_as_float(pa[c]) - Dr), p1 * (__uint_as_float(pa[c + 1]) - Dr));
-        }
-      }
-      if (t >= 1 && !wait_warp(&sm.pds_empty, (t - 1) & 1, wc)) {
-        ok = false;
-        break;
-      }
+        for (int u = 0; u < 4; ++u) {  // one 16-byte unit = 8 kv columns
+          uint32_t ph[4], pl[4], dh[4], dl[4];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        *reinterpret_cast<uint4*>(sm.p + sw128_offset(r, u)) = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2],
-                                                                         pk[4 * u + 3]);
-        *reinterpret_cast<uint4*>(sm.ds + sw128_offset(r, u)) =
-            make_uint4(dk_[4 * u], dk_[4 * u + 1], dk_[4 * u + 2], dk_[4 * u + 3]);
+          for (int e = 0; e < 4; ++e) {
+            const int c = u * 8 + 2 * e;  // column within this half
+            float p0 = fast_exp2(fmaf(__uint_as_float(sa[c]), scale_log2, -lse2));
+            float p1 = fast_exp2(fmaf(__uint_as_float(sa[c + 1]), scale_log2, -lse2));
+            if (h * 32 + c >= kv_valid) p0 = 0.f;
+            if (h * 32 + c + 1 >= kv_valid) p1 = 0.f;
+            split_bf16(p0, p1, ph[e], pl[e]);
+            split_bf16(p0 * (__uint_as_float(pa[c]) - Dr), p1 * (__uint_as_float(pa[c + 1]) - Dr), dh[e], dl[e]);
+          }
+          const uint32_t off = sw128_offset(r, h * 4 + u);
+          *reinterpret_cast<uint4*>(sm.p[0] + off) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+          *reinterpret_cast<uint4*>(sm.p[1] + off) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
+          *reinterpret_cast<uint4*>(sm.ds[0] + off) = make_uint4(dh[0], dh[1], dh[2], dh[3]);
+          *reinterpret_cast<uint4*>(sm.ds[1] + off) = make_uint4(dl[0], dl[1], dl[2], dl[3]);
+        }
       }
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&sm.pds_full);
     }
     // epilogue: dV_j = (dV^T)^T, dK_j = scale * (dK^T)^T; thread r <-> feature r
+    const long long base = ((long long)bh * N + (long long)j * 64) * D + r;
     if (n == 0) {
       // no q-block keeps kv-block j: its gradients are zero
       if (r < D) {
         for (int c = 0; c < kv_valid; ++c) {
-          const long long o = ((long long)bh * N + (long long)j * 64 + c) * D + r;
-          dv[o] = __float2bfloat16(0.f);
-          dk[o] = __float2bfloat16(0.f);
+          if (grad_f32) {
+            static_cast<float*>(dv)[base + (long long)c * D] = 0.f;
+            static_cast<float*>(dk)[base + (long long)c * D] = 0.f;
+          } else {
+            static_cast<__nv_bfloat16*>(dv)[base + (long long)c * D] = __float2bfloat16(0.f);
+            static_cast<__nv_bfloat16*>(dk)[base + (long long)c * D] = __float2bfloat16(0.f);
+          }
         }
       }
     } else if (n > 0) {
@@ -312,14 +337,23 @@ __global__ void __launch_bounds__(320, 1) bwd_kernel(const __grid_constant__ CUt
           tmem_ld32(tl + col, a);
           tmem_ld32(tl + col + 32, b);
           tmem_wait_ld();
-          __nv_bfloat16* dst = (which == 0) ? dv : dk;
+          void* dst = (which == 0) ? dv : dk;
           const float f = (which == 0) ? 1.f : scale;
           if (r < D) {
-            __nv_bfloat16* col = dst + ((long long)bh * N + (long long)j * 64) * D + r;
+            if (grad_f32) {
+              float* o = static_cast<float*>(dst) + base;
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              if (c < kv_valid) col[(long long)c * D] = __float2bfloat16(__uint_as_float(a[c]) * f);
-              if (c + 32 < kv_valid) col[(long long)(c + 32) * D] = __float2bfloat16(__uint_as_float(b[c]) * f);
+              for (int c = 0; c < 32; ++c) {
+                if (c < kv_valid) o[(long long)c * D] = __uint_as_float(a[c]) * f;
+                if (c + 32 < kv_valid) o[(long long)(c + 32) * D] = __uint_as_float(b[c]) * f;
+              }
+            } else {
+              __nv_bfloat16* o = static_cast<__nv_bfloat16*>(dst) + base;
+#pragma unroll
+              for (int c = 0; c < 32; ++c) {
+                if (c < kv_valid) o[(long long)c * D] = __float2bfloat16(__uint_as_float(a[c]) * f);
+                if (c + 32 < kv_valid) o[(long long)(c + 32) * D] = __float2bfloat16(__uint_as_float(b[c]) * f);
+              }
             }
           }
         }
@@ -335,11 +369,12 @@ __global__ void __launch_bounds__(320, 1) bwd_kernel(const __grid_constant__ CUt
   }
 }
 
-// D = rowsum(dO * O) in fp32; zero the fp32 dQ accumulator row. 16 threads per row.
+// D = rowsum(dO * (O + O_lo)) in fp32; zero the fp32 dQ row. 16 threads per row.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
+                                                      const __nv_bfloat16* __restrict__ o_lo,
                                                       const __nv_bfloat16* __restrict__ dout,
-                                                      float* __restrict__ dvec, float* __restrict__ dq_acc,
+                                                      float* __restrict__ dvec, float* __restrict__ dq32,
                                                       long long rows) {
   constexpr int TPR = 16;
   constexpr int EPT = D / TPR;  // 8 (d=128) or 4 (d=64) elements per thread
@@ -347,21 +382,25 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __res
   const int tc = threadIdx.x % TPR;
   float acc = 0.f;
   if (row < rows) {
-    const __nv_bfloat16* po = o + row * D + tc * EPT;
-    const __nv_bfloat16* pd = dout + row * D + tc * EPT;
+    const long long off = row * D + tc * EPT;
 #pragma unroll
     for (int e = 0; e < EPT; e += 2) {
-      const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(po + e));
-      const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(pd + e));
+      float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(o + off + e));
+      if (o_lo) {
+        const float2 l = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(o_lo + off + e));
+        a.x += l.x;
+        a.y += l.y;
+      }
+      const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(dout + off + e));
       acc = fmaf(a.x, b.x, acc);
       acc = fmaf(a.y, b.y, acc);
     }
-    float4* z = reinterpret_cast<float4*>(dq_acc + row * D + tc * EPT);
+    float4* z = reinterpret_cast<float4*>(dq32 + off);
 #pragma unroll
     for (int e = 0; e < EPT / 4; ++e) z[e] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
 #pragma unroll
-  for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffff, acc, off);
+  for (int s = TPR / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffff, acc, s);
   if (row < rows && tc == 0) dvec[row] = acc;
 }
 
@@ -375,15 +414,16 @@ __global__ void __launch_bounds__(256) dq_convert_kernel(const float4* __restric
 
 cudaError_t launch_bwd(const BwdArgs& a, int d, cudaStream_t s) {
   const long long rows = (long long)a.BH * a.N;
-  // 1. D and dQ accumulator reset
+  float* dq32 = a.grad_f32 ? static_cast<float*>(a.dq) : a.dq_acc;
+  // 1. D and dQ reset
   {
     dim3 grid((unsigned)((rows + 15) / 16));
     if (d == 128)
-      bwd_pre_kernel<128><<<grid, 256, 0, s>>>((const __nv_bfloat16*)a.o, (const __nv_bfloat16*)a.dout, a.dvec,
-                                               a.dq_acc, rows);
+      bwd_pre_kernel<128><<<grid, 256, 0, s>>>((const __nv_bfloat16*)a.o, (const __nv_bfloat16*)a.o_lo,
+                                               (const __nv_bfloat16*)a.dout, a.dvec, dq32, rows);
     else
-      bwd_pre_kernel<64><<<grid, 256, 0, s>>>((const __nv_bfloat16*)a.o, (const __nv_bfloat16*)a.dout, a.dvec,
-                                              a.dq_acc, rows);
+      bwd_pre_kernel<64><<<grid, 256, 0, s>>>((const __nv_bfloat16*)a.o, (const __nv_bfloat16*)a.o_lo,
+                                              (const __nv_bfloat16*)a.dout, a.dvec, dq32, rows);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -395,26 +435,27 @@ cudaError_t launch_bwd(const BwdArgs& a, int d, cudaStream_t s) {
       cudaError_t e = cudaFuncSetAttribute(bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
       bwd_kernel<128><<<grid, 320, smem, s>>>(*a.tm_q, *a.tm_k, *a.tm_v, *a.tm_do, a.lse, a.dvec, a.col_cnt,
-                                              a.col_idx, a.dq_acc, (__nv_bfloat16*)a.dk, (__nv_bfloat16*)a.dv, a.N,
-                                              a.Tm, a.Tn, a.scale, a.scale_log2, a.status, a.wait_limit_ns);
+                                              a.col_idx, dq32, a.dk, a.dv, a.grad_f32, a.N, a.Tm, a.Tn, a.scale,
+                                              a.scale_log2, a.status, a.wait_limit_ns);
     } else {
       const size_t smem = sizeof(BwdSmem<64>) + 1024;
       cudaError_t e = cudaFuncSetAttribute(bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
       bwd_kernel<64><<<grid, 320, smem, s>>>(*a.tm_q, *a.tm_k, *a.tm_v, *a.tm_do, a.lse, a.dvec, a.col_cnt,
-                                             a.col_idx, a.dq_acc, (__nv_bfloat16*)a.dk, (__nv_bfloat16*)a.dv, a.N,
-                                             a.Tm, a.Tn, a.scale, a.scale_log2, a.status, a.wait_limit_ns);
+                                             a.col_idx, dq32, a.dk, a.dv, a.grad_f32, a.N, a.Tm, a.Tn, a.scale,
+                                             a.scale_log2, a.status, a.wait_limit_ns);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   // 3. dQ fp32 -> bf16
-  {
+  if (!a.grad_f32) {
     const long long n4 = rows * d / 4;
     const unsigned blocks = (unsigned)std::min<long long>((n4 + 255) / 256, 148LL * 16);
     dq_convert_kernel<<<blocks, 256, 0, s>>>((const float4*)a.dq_acc, (uint2*)a.dq, n4);
     return cudaGetLastError();
   }
+  return cudaSuccess;
 }
 
 }  // namespace spa2

@@ -6,18 +6,21 @@
 // kv-blocks j (b_kv = 64 rows each) listed in the CSR row of i.
 //
 //   warp 4      TMA producer: Q_i once, then K_j / V_j through a 2-slot ring.
-//   warp 5      MMA issuer (one thread): S = Q K_j^T (SS, M=128 N=64 K=d) into
-//               one of two TMEM S buffers; O += P V_j (TS: P from TMEM,
-//               M=128 N=d K=64). Owns the 256-column TMEM allocation.
+//   warp 5      MMA issuer (one thread): S = Q K_j^T (SS, bf16, M=128 N=64 K=d)
+//               into one of two TMEM S buffers; O += P V_j (TS: P from TMEM,
+//               fp16 operands, M=128 N=d K=64). Owns the 256-column TMEM
+//               allocation.
 //   warps 0-3   softmax, thread t <-> query row t <-> TMEM lane t: load S,
-//               online max / exp2 / sum in registers, write P (bf16) over the
-//               S buffer, rescale O in TMEM only when the running max grew by
+//               online max / exp2 / sum in registers, write P (fp16, values in
+//               [0, 256]: 8x finer rounding than bf16) over the S buffer, rescale O in TMEM only when the running max grew by
 //               more than 2^8 (lazy rescale), then the epilogue O / l -> bf16
-//               -> smem -> TMA store, and LSE.
+//               (and optionally its bf16 residual) -> smem -> TMA store, LSE.
 //
 // TMEM columns: [0,64) S/P buffer 0, [64,128) S/P buffer 1, [128,128+d) O.
-// Shared memory: Q 128 x d bf16 (reused as the O staging tile), 2 x (K, V)
-// 64 x d bf16; every tile in 128-byte-swizzled 64-column chunks as TMA writes
+// v_to_f16_kernel  fp16 copy of V for the P V product (exact for bf16 values
+//               of magnitude <= 65504; larger ones are clamped and reported).
+// Shared memory: Q 128 x d bf16 (reused as the O staging tile), 2 x (K bf16,
+// V fp16) 64 x d; every tile in 128-byte-swizzled 64-column chunks as TMA writes
 // them. Two CTAs fit on one SM (TMEM 2 x 256 columns, smem 2 x ~97 KB), so one
 // CTA's softmax overlaps the other's MMAs.
 #include "common.cuh"
@@ -54,12 +57,13 @@ __global__ void __launch_bounds__(192, 2) fwd_kernel(const __grid_constant__ CUt
                                                      const __grid_constant__ CUtensorMap tm_k,
                                                      const __grid_constant__ CUtensorMap tm_v,
                                                      const __grid_constant__ CUtensorMap tm_o,
+                                                     const __grid_constant__ CUtensorMap tm_olo, int has_olo,
                                                      const int* __restrict__ row_cnt, const int* __restrict__ row_idx,
                                                      float* __restrict__ lse, int N, int Tm, int Tn, float scale_log2,
                                                      int* status, unsigned long long wait_limit_ns) {
   constexpr int CH = D / 64;
   constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, false, false);
-  constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, false, true);
+  constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, false, true, /*f16=*/true);
   constexpr uint32_t Q_BYTES = 128 * D * 2;
   constexpr uint32_t KV_BYTES = 64 * D * 2;
 
@@ -227,8 +231,8 @@ __global__ void __launch_bounds__(192, 2) fwd_kernel(const __grid_constant__ CUt
         const float p2 = fast_exp2(fmaf(__uint_as_float(rb[2 * c]), scale_log2, neg_m));
         const float p3 = fast_exp2(fmaf(__uint_as_float(rb[2 * c + 1]), scale_log2, neg_m));
         rs += (p0 + p1) + (p2 + p3);
-        pk[c] = pack_bf16(p0, p1);
-        pk[16 + c] = pack_bf16(p2, p3);
+        pk[c] = pack_f16(p0, p1);
+        pk[16 + c] = pack_f16(p2, p3);
       }
       l += rs;
       tmem_st32(tl + s * 64, pk);
@@ -268,16 +272,25 @@ __global__ void __launch_bounds__(192, 2) fwd_kernel(const __grid_constant__ CUt
         uint32_t ov[32];
         tmem_ld32(tl + 128 + cc * 32, ov);
         tmem_wait_ld();
-        uint32_t pk[16];
+        uint32_t hi[16], lo[16];
 #pragma unroll
-        for (int c = 0; c < 16; ++c)
-          pk[c] = pack_bf16(__uint_as_float(ov[2 * c]) * inv_l, __uint_as_float(ov[2 * c + 1]) * inv_l);
-        uint8_t* chunk = sm.q[cc >> 1];
+        for (int c = 0; c < 16; ++c) {
+          const float a = __uint_as_float(ov[2 * c]) * inv_l, b = __uint_as_float(ov[2 * c + 1]) * inv_l;
+          hi[c] = pack_bf16(a, b);
+          const float2 hf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hi[c]));
+          lo[c] = pack_bf16(a - hf.x, b - hf.y);
+        }
         const uint32_t u0 = (cc & 1) * 4;
+        uint8_t* chunk = sm.q[cc >> 1];
+        uint8_t* chunk_lo = &sm.k[0][0][0] + (cc >> 1) * (128 * 128);  // K/V ring is free now
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
+        for (int e = 0; e < 4; ++e) {
           *reinterpret_cast<uint4*>(chunk + sw128_offset(r, u0 + e)) =
-              make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+              make_uint4(hi[4 * e], hi[4 * e + 1], hi[4 * e + 2], hi[4 * e + 3]);
+          if (has_olo)
+            *reinterpret_cast<uint4*>(chunk_lo + sw128_offset(r, u0 + e)) =
+                make_uint4(lo[4 * e], lo[4 * e + 1], lo[4 * e + 2], lo[4 * e + 3]);
+        }
       }
       const long long row = (long long)i * 128 + r;
       if (row < N) lse[(long long)bh * N + row] = (m_use + log2f(l)) * 0.69314718055994530942f;
@@ -286,6 +299,8 @@ __global__ void __launch_bounds__(192, 2) fwd_kernel(const __grid_constant__ CUt
     named_bar_sync(1, 128);
     if (threadIdx.x == 0 && sm.epi_ok) {
       for (int c = 0; c < CH; ++c) tma_store_3d(&tm_o, sm.q[c], c * 64, i * 128, bh);
+      if (has_olo)
+        for (int c = 0; c < CH; ++c) tma_store_3d(&tm_olo, &sm.k[0][0][0] + c * (128 * 128), c * 64, i * 128, bh);
       tma_store_commit();
       tma_store_wait_all();
     }
@@ -299,19 +314,50 @@ __global__ void __launch_bounds__(192, 2) fwd_kernel(const __grid_constant__ CUt
   }
 }
 
+// bf16 -> fp16 copy of V (16 bytes per thread and step); |v| > 65504 is clamped
+// to the largest finite fp16 and reported as SPA2_ERR_RANGE.
+__global__ void __launch_bounds__(256) v_to_f16_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                                       long long n8, int* status) {
+  bool bad = false;
+  for (long long e = (long long)blockIdx.x * 256 + threadIdx.x; e < n8; e += (long long)gridDim.x * 256) {
+    const uint4 v = src[e];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+      if (!(fabsf(f.x) <= 65504.f) || !(fabsf(f.y) <= 65504.f)) {
+        bad = true;
+        f.x = fminf(fmaxf(f.x, -65504.f), 65504.f);
+        f.y = fminf(fmaxf(f.y, -65504.f), 65504.f);
+      }
+      o[i] = pack_f16(f.x, f.y);
+    }
+    dst[e] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  if (bad) report(status, SPA2_ERR_RANGE);
+}
+
+cudaError_t launch_v_to_f16(const void* v, void* v16, long long elems, int* status, cudaStream_t s) {
+  const long long n8 = elems / 8;
+  const unsigned blocks = (unsigned)((n8 + 255) / 256 < 148LL * 32 ? (n8 + 255) / 256 : 148LL * 32);
+  v_to_f16_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4*>(v), static_cast<uint4*>(v16), n8, status);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_fwd(const FwdArgs& a, int d, cudaStream_t s) {
   dim3 grid(a.Tm, a.BH);
   if (d == 128) {
     const size_t smem = sizeof(FwdSmem<128>) + 1024;
     cudaError_t e = cudaFuncSetAttribute(fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    fwd_kernel<128><<<grid, 192, smem, s>>>(*a.tm_q, *a.tm_k, *a.tm_v, *a.tm_o, a.row_cnt, a.row_idx, a.lse, a.N,
+    fwd_kernel<128><<<grid, 192, smem, s>>>(*a.tm_q, *a.tm_k, *a.tm_v, *a.tm_o, *a.tm_olo, a.has_olo, a.row_cnt, a.row_idx, a.lse, a.N,
                                             a.Tm, a.Tn, a.scale_log2, a.status, a.wait_limit_ns);
   } else {
     const size_t smem = sizeof(FwdSmem<64>) + 1024;
     cudaError_t e = cudaFuncSetAttribute(fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    fwd_kernel<64><<<grid, 192, smem, s>>>(*a.tm_q, *a.tm_k, *a.tm_v, *a.tm_o, a.row_cnt, a.row_idx, a.lse, a.N,
+    fwd_kernel<64><<<grid, 192, smem, s>>>(*a.tm_q, *a.tm_k, *a.tm_v, *a.tm_o, *a.tm_olo, a.has_olo, a.row_cnt, a.row_idx, a.lse, a.N,
                                            a.Tm, a.Tn, a.scale_log2, a.status, a.wait_limit_ns);
   }
   return cudaGetLastError();

@@ -7,6 +7,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -226,11 +227,13 @@ SPA2_DEV uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   return d;
 }
 
-// Instruction descriptor of kind::f16 with bf16 A/B and fp32 accumulation.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
+// Instruction descriptor of kind::f16 with fp32 accumulation; A and B are both
+// bf16 (default) or both fp16 (f16 = true).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major, bool b_mn_major,
+                                                      bool f16 = false) {
   return (1u << 4)                                // D format: f32
-         | (1u << 7)                              // A format: bf16
-         | (1u << 10)                             // B format: bf16
+         | ((f16 ? 0u : 1u) << 7)                 // A format: f16 = 0, bf16 = 1
+         | ((f16 ? 0u : 1u) << 10)                // B format: f16 = 0, bf16 = 1
          | ((a_mn_major ? 1u : 0u) << 15)         // A major
          | ((b_mn_major ? 1u : 0u) << 16)         // B major
          | (static_cast<uint32_t>(N >> 3) << 17)  // N / 8
@@ -239,6 +242,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
 
 // byte offset of 16-byte unit `u` of row `r` in a 128-byte-swizzled tile (tile base 1024-aligned)
 SPA2_DEV uint32_t sw128_offset(uint32_t r, uint32_t u) { return r * 128u + ((u ^ (r & 7u)) << 4); }
+
+SPA2_DEV uint32_t pack_f16(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);  // .x = lo (low 16 bits), .y = hi
+  return *reinterpret_cast<uint32_t*>(&v);
+}
 
 SPA2_DEV uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low 16 bits), .y = hi

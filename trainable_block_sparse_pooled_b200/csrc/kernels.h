@@ -30,8 +30,10 @@ cudaError_t launch_csc(const uint32_t* bits, int BH, int Tm, int Tn, int W, int*
 struct FwdArgs {
   const CUtensorMap* tm_q;   // box {64, 128, 1}
   const CUtensorMap* tm_k;   // box {64, 64, 1}
-  const CUtensorMap* tm_v;   // box {64, 64, 1}
+  const CUtensorMap* tm_v;   // box {64, 64, 1}, fp16 copy of V
   const CUtensorMap* tm_o;   // box {64, 128, 1}
+  const CUtensorMap* tm_olo; // box {64, 128, 1}; O residual, used when has_olo
+  int has_olo;
   const int* row_cnt;
   const int* row_idx;
   float* lse;
@@ -41,6 +43,7 @@ struct FwdArgs {
   unsigned long long wait_limit_ns;
 };
 cudaError_t launch_fwd(const FwdArgs& a, int d, cudaStream_t s);
+cudaError_t launch_v_to_f16(const void* v, void* v16, long long elems, int* status, cudaStream_t s);
 
 // attn_bwd.cu
 struct BwdArgs {
@@ -49,6 +52,7 @@ struct BwdArgs {
   const CUtensorMap* tm_v;    // box {64, 64, 1}
   const CUtensorMap* tm_do;   // box {64, 128, 1}
   const void* o;
+  const void* o_lo;   // may be null
   const void* dout;
   const float* lse;
   const int* col_cnt;
@@ -58,6 +62,7 @@ struct BwdArgs {
   void* dq;
   void* dk;
   void* dv;
+  int grad_f32;       // 1: dq/dk/dv are fp32 (dQ accumulates in place), 0: bf16
   int BH, N, Tm, Tn;
   float scale;        // softmax_scale
   float scale_log2;   // softmax_scale * log2(e)
