@@ -19,5 +19,6 @@ from .spa2_oracle import (  # noqa: F401
     masked_attn_fwd_rows,
     masked_attn_bwd,
     masked_attn_bwd_blocks,
+    masked_attn_bwd_rows,
     attn_flops,
 )

@@ -286,6 +286,33 @@ def masked_attn_bwd_blocks(Q, K, V, mask, dO, bq: int, bkv: int, scale, b: int, 
     return dQ, dKV
 
 
+def masked_attn_bwd_rows(Q, K, V, mask, dO, bq: int, bkv: int, scale, b: int, h: int, qblocks):
+    """Backward contributions of the q-blocks ``qblocks`` of head (b, h).
+
+    Returns ({i: dQ_i}, dK_part, dV_part) where dK_part / dV_part [N, d] hold
+    the sums over the listed q-blocks only (the full dK, dV sum every q-block).
+    """
+    N = Q.shape[-2]
+    Kh = np.asarray(K[b, h], dtype=np.float64)
+    Vh = np.asarray(V[b, h], dtype=np.float64)
+    dQ = {}
+    dKp = np.zeros((N, K.shape[-1]))
+    dVp = np.zeros((N, V.shape[-1]))
+    for i in qblocks:
+        lo, hi = i * bq, min(N, (i + 1) * bq)
+        Qi = np.asarray(Q[b, h, lo:hi], dtype=np.float64)
+        dOi = np.asarray(dO[b, h, lo:hi], dtype=np.float64)
+        cols = _kept_cols(mask[b, h, i], N, bkv)
+        P, _ = _row_block_softmax(Qi, Kh[cols], scale)
+        dVp[cols] += P.T @ dOi
+        dP = dOi @ Vh[cols].T
+        D = (P * dP).sum(axis=1, keepdims=True)
+        dS = P * (dP - D)
+        dQ[i] = (dS @ Kh[cols]) * scale
+        dKp[cols] += (dS.T @ Qi) * scale
+    return dQ, dKp, dVp
+
+
 def attn_flops(mask, N: int, bq: int, bkv: int, d: int) -> float:
     """Forward flops 4*d*sum over kept (i, j) of valid q rows x valid kv cols."""
     mask = np.asarray(mask, dtype=bool)

@@ -1,0 +1,28 @@
+"""Host-side logic that needs no GPU: sparsity calibration (against the oracle's
+mask as the counting function) and the bench's flop / byte accounting."""
+
+import numpy as np
+
+import oracle
+from trainable_block_sparse_pooled_b200 import calibrate, synth
+
+
+def test_calibration_hits_target_with_oracle_counts():
+    q, k, _ = synth.smoothed_field(B=1, H=2, N=8192, d=64, seed=0, grid=(8, 32, 32))
+    Qb = oracle.pool_blocks(q.float().numpy().astype(np.float64), 128)
+    Kb = oracle.pool_blocks(k.float().numpy().astype(np.float64), 64)
+    pbar32 = oracle.pooled_attention(Qb, Kb, 64).astype(np.float32)
+    total = pbar32.shape[0] * pbar32.shape[1] * pbar32.shape[2] * pbar32.shape[3]
+
+    def kept(kf, pf):
+        return int(oracle.select_blocks(pbar32, kf, pf).sum())
+
+    kf, pf, s = calibrate.calibrate_p(kept, total, 0.90, tol=0.01)
+    assert abs(kf - 0.05) < 1e-12
+    assert abs(s - 0.90) <= 0.01
+    assert abs((1 - kept(kf, pf) / total) - s) < 1e-12
+
+
+def test_calibration_returns_topk_only_when_target_is_loose():
+    kf, pf, s = calibrate.calibrate_p(lambda k, p: 10, 100, 0.95)
+    assert pf == 0.0 and abs(s - 0.9) < 1e-12

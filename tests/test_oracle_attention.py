@@ -145,3 +145,18 @@ def test_sampled_backward_matches_full_backward():
     for j, (gk, gv) in skv.items():
         np.testing.assert_allclose(gk, dK[0, 1, j * 64:j * 64 + gk.shape[0]], atol=1e-12)
         np.testing.assert_allclose(gv, dV[0, 1, j * 64:j * 64 + gv.shape[0]], atol=1e-12)
+
+
+def test_row_contributions_sum_to_full_backward():
+    Q, K, V, dO = _inputs(12, N=400)
+    B, H, N, d = Q.shape
+    Tm, Tn = oracle.block_counts(N, 128, 64)
+    mask = _random_mask(12, B, H, Tm, Tn, 0.5)
+    scale = 1 / math.sqrt(d)
+    dQ, dK, dV = oracle.masked_attn_bwd(Q, K, V, mask, dO, 128, 64)
+    q1, k1, v1 = oracle.masked_attn_bwd_rows(Q, K, V, mask, dO, 128, 64, scale, 0, 1, [0, 2])
+    q2, k2, v2 = oracle.masked_attn_bwd_rows(Q, K, V, mask, dO, 128, 64, scale, 0, 1, [1, 3])
+    np.testing.assert_allclose(k1 + k2, dK[0, 1], atol=1e-12)
+    np.testing.assert_allclose(v1 + v2, dV[0, 1], atol=1e-12)
+    for i, g in {**q1, **q2}.items():
+        np.testing.assert_allclose(g, dQ[0, 1, i * 128:i * 128 + g.shape[0]], atol=1e-12)

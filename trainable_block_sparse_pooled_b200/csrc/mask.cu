@@ -13,10 +13,10 @@
 // id asc); Top-k keeps the first K ranks; Top-p keeps rank r while the
 // quantised mass floor(2^32 P) of ranks before r is below floor(2^32 p). Both
 // are prefixes of the same order, so the union is the first max(K, R) ranks.
-// Instead of sorting, each warp runs a 4-pass radix search (8 bits per pass)
-// over the float bit patterns (monotone for P >= 0): once weighted by counts
-// (the K-th largest value) and once by masses (the value where the running
-// mass reaches p), then resolves ties at the boundary by block id.
+// Instead of sorting, each warp bisects the float bit patterns (monotone for
+// P >= 0): once weighted by counts (the K-th largest value) and, when the
+// Top-k set does not already reach p, once by masses (the value where the
+// running mass reaches p); ties at the boundary go by ascending block id.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -93,151 +93,103 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
 
 // ---------------------------------------------------------------------------
 // warp-level exact hybrid selection on one float32 P-bar row held in smem
+//
+// Keys are the float bit patterns (monotone for P >= 0). Masses are the exact
+// integers q_j = floor(2^32 P_j) held as doubles (a row's total stays below
+// 2^53, so every sum is exact). Two bisections over the key space, each ~30
+// warp passes with no atomics:
+//   Top-k: largest T with count(key >= T) >= K  -> K-th largest value T_K;
+//   Top-p: largest T with mass(key >= T) >= thr -> value of the last block the
+//          inclusive walk keeps (only needed when the Top-k set's mass < thr).
+// Ties at the boundary value are resolved by ascending block id.
 // ---------------------------------------------------------------------------
-struct WarpHist {
-  unsigned long long w[256];
-  uint32_t c[256];
-};
+SPA2_DEV double mass_of(float p) { return floor((double)p * 4294967296.0); }
 
-struct RadixResult {
-  uint32_t value;              // bit pattern of the boundary value T
-  unsigned long long gt_w;     // weight of elements with bits > T
-  uint32_t gt_c;               // count of elements with bits > T
-  uint32_t eq_c;               // count of elements with bits == T
-};
-
-SPA2_DEV unsigned long long quant_mass(float p) {
-  // floor(2^32 * p) for p in [0, 1]: the product is exact (power-of-two scale)
-  return __float2ull_rz(p * 4294967296.0f);
+SPA2_DEV double warp_sum_d(double x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffff, x, o);
+  return x;
 }
 
-// Largest bit pattern T with weight(bits >= T) >= target, where weight is the
-// element count (BY_MASS = false) or the quantised mass (BY_MASS = true).
-// Requires weight(all) >= target > 0.
-template <bool BY_MASS>
-SPA2_DEV RadixResult radix_search(const float* row, int Tn, unsigned long long target, WarpHist* h) {
-  const uint32_t lane = lane_id();
-  uint32_t prefix = 0;
-  unsigned long long acc_w = 0;
-  uint32_t acc_c = 0;
-  uint32_t eq_c = 0;
-#pragma unroll 1
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int b = lane; b < 256; b += 32) {
-      h->w[b] = 0ull;
-      h->c[b] = 0u;
-    }
-    __syncwarp();
-    const uint32_t hi_mask = (shift == 24) ? 0u : (0xFFFFFFFFu << (shift + 8));
-    for (int j = lane; j < Tn; j += 32) {
-      const float p = row[j];
-      const uint32_t u = __float_as_uint(p);
-      if ((u & hi_mask) == prefix) {
-        const uint32_t dg = (u >> shift) & 0xFFu;
-        atomicAdd(&h->c[dg], 1u);
-        atomicAdd(&h->w[dg], BY_MASS ? quant_mass(p) : 1ull);
-      }
-    }
-    __syncwarp();
-    // lane l owns digits 255-8l .. 248-8l (descending)
-    unsigned long long lw = 0;
-    uint32_t lc = 0;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      lw += h->w[255 - 8 * lane - e];
-      lc += h->c[255 - 8 * lane - e];
-    }
-    unsigned long long ex_w = lw;  // inclusive scan, made exclusive below
-    uint32_t ex_c = lc;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      unsigned long long tw = __shfl_up_sync(0xffffffff, ex_w, o);
-      uint32_t tc = __shfl_up_sync(0xffffffff, ex_c, o);
-      if (lane >= (uint32_t)o) {
-        ex_w += tw;
-        ex_c += tc;
-      }
-    }
-    ex_w -= lw;
-    ex_c -= lc;
-    const bool reach = acc_w + ex_w + lw >= target;
-    const uint32_t bal = __ballot_sync(0xffffffff, reach);
-    const int fl = __ffs(bal) - 1;  // exists: total weight >= target
-    uint32_t dg = 0, nc = 0, ec = 0;
-    unsigned long long nw = 0;
-    if ((int)lane == fl) {
-      unsigned long long cw = acc_w + ex_w;
-      uint32_t cc = acc_c + ex_c;
-#pragma unroll 1
-      for (int e = 0; e < 8; ++e) {
-        const int d = 255 - 8 * (int)lane - e;
-        if (cw + h->w[d] >= target) {
-          dg = d;
-          ec = h->c[d];
-          break;
-        }
-        cw += h->w[d];
-        cc += h->c[d];
-      }
-      nw = cw;
-      nc = cc;
-    }
-    dg = __shfl_sync(0xffffffff, dg, fl);
-    acc_w = __shfl_sync(0xffffffff, nw, fl);
-    acc_c = __shfl_sync(0xffffffff, nc, fl);
-    eq_c = __shfl_sync(0xffffffff, ec, fl);
-    prefix |= dg << shift;
-    __syncwarp();
+struct Boundary {
+  uint32_t gt_c;  // elements with key > T
+  uint32_t eq_c;  // elements with key == T
+  double gt_m;    // their mass
+  double all_m;   // mass of the whole row
+};
+
+SPA2_DEV Boundary boundary_stats(const uint32_t* keys, const double* qm, int Tn, uint32_t T) {
+  uint32_t gt = 0, eq = 0;
+  double gm = 0.0, am = 0.0;
+  for (int j = lane_id(); j < Tn; j += 32) {
+    const uint32_t u = keys[j];
+    const double q = qm[j];
+    gt += (u > T);
+    eq += (u == T);
+    gm += (u > T) ? q : 0.0;
+    am += q;
   }
-  return RadixResult{prefix, acc_w, acc_c, eq_c};
+  return Boundary{__reduce_add_sync(0xffffffff, gt), __reduce_add_sync(0xffffffff, eq), warp_sum_d(gm), warp_sum_d(am)};
 }
 
-// Select the kept blocks of one row and write its CSR entry, kept-bit words
-// and optional uint8 bitmap. `row` is the float32 P-bar row in shared memory.
-SPA2_DEV void select_row_warp(const float* row, int Tn, int K, unsigned long long thr, WarpHist* h,
+// Select the kept blocks of one row; write its CSR entry, kept-bit words and
+// optional uint8 bitmap. `keys` = float bits of the P-bar row, `qm` = masses.
+SPA2_DEV void select_row_warp(const uint32_t* keys, const double* qm, int Tn, int K, double thr,
                               int* row_cnt_out, int* row_idx_out, uint32_t* bits_out, uint8_t* bitmap_out,
                               int* status) {
   const uint32_t lane = lane_id();
-  // Top-k boundary
-  const RadixResult rk = radix_search<false>(row, Tn, (unsigned long long)K, h);
-  const uint32_t tK = (uint32_t)K - rk.gt_c;
-  // Top-p count R
-  int R = 0;
-  RadixResult rp{0u, 0ull, 0u, 0u};
-  uint32_t tR = 0;
-  if (thr > 0) {
-    unsigned long long tot = 0;
-    for (int j = lane; j < Tn; j += 32) tot += quant_mass(row[j]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffff, tot, o);
-    if (tot < thr) {
-      R = Tn;
+  // ---- Top-k boundary: largest T with count(key >= T) >= K (K <= Tn)
+  uint32_t lo = 0u, hi = 0x3F800001u;  // count(0) = Tn >= K; nothing exceeds 1.0f
+#pragma unroll 1
+  while (hi - lo > 1u) {
+    const uint32_t mid = lo + ((hi - lo) >> 1);
+    uint32_t c = 0;
+    for (int j = lane; j < Tn; j += 32) c += (keys[j] >= mid);
+    c = __reduce_add_sync(0xffffffff, c);
+    if (c >= (uint32_t)K) lo = mid; else hi = mid;
+  }
+  const uint32_t TK = lo;
+  const Boundary bk = boundary_stats(keys, qm, Tn, TK);
+  const uint32_t tK = (uint32_t)K - bk.gt_c;          // tied blocks Top-k takes at T_K
+  const double massK = bk.gt_m + (double)tK * mass_of(__uint_as_float(TK));
+
+  // ---- Top-p: R <= K iff the first K ranks already reach thr
+  uint32_t bv = TK, bt = tK;
+  bool keep_all = (K >= Tn);
+  int n = K;
+  if (!keep_all && thr > 0.0 && massK < thr) {
+    if (bk.all_m < thr) {
+      keep_all = true;                                  // every rank stays below thr
+      n = Tn;
     } else {
-      rp = radix_search<true>(row, Tn, thr, h);
-      const unsigned long long need = thr - rp.gt_w;  // > 0
-      const unsigned long long qv = quant_mass(__uint_as_float(rp.value));  // > 0 here
-      unsigned long long ties = (need + qv - 1) / qv;
-      tR = (uint32_t)min((unsigned long long)rp.eq_c, ties);
-      R = (int)(rp.gt_c + tR);
+      lo = 0u;                                          // mass(key >= 0) = all >= thr
+      hi = TK + 1u;                                     // mass(key > T_K) <= massK < thr
+#pragma unroll 1
+      while (hi - lo > 1u) {
+        const uint32_t mid = lo + ((hi - lo) >> 1);
+        double m = 0.0;
+        for (int j = lane; j < Tn; j += 32) m += (keys[j] >= mid) ? qm[j] : 0.0;
+        m = warp_sum_d(m);
+        if (m >= thr) lo = mid; else hi = mid;
+      }
+      const Boundary bp = boundary_stats(keys, qm, Tn, lo);
+      const double need = thr - bp.gt_m;               // > 0
+      const double qv = mass_of(__uint_as_float(lo));  // > 0 here
+      const double ties = ceil(need / qv);             // exact: integers below 2^53
+      bv = lo;
+      bt = (uint32_t)fmin((double)bp.eq_c, ties);
+      n = (int)(bp.gt_c + bt);
+      keep_all = (n >= Tn);
     }
   }
-  const int n = max(K, R);
-  const bool keep_all = (n >= Tn);
-  uint32_t bv, bt;
-  if (R > K) {
-    bv = rp.value;
-    bt = tR;
-  } else {
-    bv = rk.value;
-    bt = tK;
-  }
+  // ---- emit ascending ids: key > bv, or key == bv among the first bt by id
   const uint32_t lt = (1u << lane) - 1u;
   int running = 0;
   uint32_t ties_seen = 0;
   for (int base = 0; base < Tn; base += 32) {
     const int j = base + (int)lane;
     const bool valid = j < Tn;
-    const uint32_t u = valid ? __float_as_uint(row[j]) : 0u;
+    const uint32_t u = valid ? keys[j] : 0u;
     const bool is_tie = valid && (u == bv);
     const uint32_t tie_bal = __ballot_sync(0xffffffff, is_tie);
     const uint32_t tie_rank = ties_seen + __popc(tie_bal & lt);
@@ -256,29 +208,30 @@ SPA2_DEV void select_row_warp(const float* row, int Tn, int K, unsigned long lon
 }
 
 // ---------------------------------------------------------------------------
-// pooled softmax + selection: ROWS q-block rows of one head per CTA (8 warps)
+// pooled softmax + selection: ROWS q-block rows of one head per CTA, one warp per
+// row; Kbar is read once per CTA (ROWS dot products per Kbar row and thread)
 // ---------------------------------------------------------------------------
 template <int D, int ROWS>
-__global__ void __launch_bounds__(256) pbar_select_kernel(const float* __restrict__ qbar,
-                                                          const float* __restrict__ kbar, int Tm, int Tn,
-                                                          float inv_sqrt_d, int K, unsigned long long thr,
-                                                          MaskOut out, uint32_t* __restrict__ bits, int W,
-                                                          int* status) {
+__global__ void __launch_bounds__(ROWS * 32) pbar_select_kernel(const float* __restrict__ qbar,
+                                                                const float* __restrict__ kbar, int Tm, int Tn,
+                                                                float inv_sqrt_d, int K, double thr, MaskOut out,
+                                                                uint32_t* __restrict__ bits, int W, int* status) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  float* qb = reinterpret_cast<float*>(smem_raw);                 // [ROWS][D]
-  float* logits = qb + ROWS * D;                                   // [ROWS][Tn]
-  WarpHist* hist = reinterpret_cast<WarpHist*>(logits + ROWS * Tn + ((ROWS * Tn) & 1));  // [8]
+  double* qm = reinterpret_cast<double*>(smem_raw);                // [ROWS][Tn] masses
+  float* qb = reinterpret_cast<float*>(qm + (size_t)ROWS * Tn);    // [ROWS][D]
+  float* prow = qb + ROWS * D;                                     // [ROWS][Tn] logits -> P-bar
+  constexpr int NT = ROWS * 32;
 
   const long long bh = blockIdx.y;
   const int i0 = blockIdx.x * ROWS;
-  for (int e = threadIdx.x; e < ROWS * D; e += 256) {
+  for (int e = threadIdx.x; e < ROWS * D; e += NT) {
     const int r = e / D;
     qb[e] = (i0 + r < Tm) ? qbar[(bh * Tm + i0 + r) * D + (e % D)] : 0.f;
   }
   __syncthreads();
 
   // logits[r][c] = Qbar_r . Kbar_c / sqrt(d), fp32, sequential over d
-  for (int c = threadIdx.x; c < Tn; c += 256) {
+  for (int c = threadIdx.x; c < Tn; c += NT) {
     float acc[ROWS];
 #pragma unroll
     for (int r = 0; r < ROWS; ++r) acc[r] = 0.f;
@@ -296,58 +249,62 @@ __global__ void __launch_bounds__(256) pbar_select_kernel(const float* __restric
       }
     }
 #pragma unroll
-    for (int r = 0; r < ROWS; ++r) logits[r * Tn + c] = acc[r] * inv_sqrt_d;
+    for (int r = 0; r < ROWS; ++r) prow[r * Tn + c] = acc[r] * inv_sqrt_d;
   }
   __syncthreads();
 
   const int w = threadIdx.x >> 5;
   const uint32_t lane = lane_id();
-  for (int r = w; r < ROWS; r += 8) {
-    const int i = i0 + r;
-    if (i >= Tm) break;
-    float* row = logits + r * Tn;
-    float m = -INFINITY;
-    for (int j = lane; j < Tn; j += 32) m = fmaxf(m, row[j]);
+  const int i = i0 + w;
+  if (i >= Tm) return;
+  float* row = prow + (size_t)w * Tn;
+  double* rq = qm + (size_t)w * Tn;
+  float m = -INFINITY;
+  for (int j = lane; j < Tn; j += 32) m = fmaxf(m, row[j]);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffff, m, o));
-    float s = 0.f;
-    for (int j = lane; j < Tn; j += 32) {
-      const float e = expf(row[j] - m);
-      row[j] = e;
-      s += e;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffff, s, o);
-    const long long rowid = bh * Tm + i;
-    for (int j = lane; j < Tn; j += 32) {
-      const float p = row[j] / s;
-      row[j] = p;
-      if (out.pbar) out.pbar[rowid * Tn + j] = p;
-    }
-    __syncwarp();
-    select_row_warp(row, Tn, K, thr, hist + w, out.row_cnt + rowid, out.row_idx + rowid * Tn, bits + rowid * W,
-                    out.bitmap ? out.bitmap + rowid * Tn : nullptr, status);
-    __syncwarp();
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffff, m, o));
+  float ssum = 0.f;
+  for (int j = lane; j < Tn; j += 32) {
+    const float e = expf(row[j] - m);
+    row[j] = e;
+    ssum += e;
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ssum += __shfl_xor_sync(0xffffffff, ssum, o);
+  const long long rowid = bh * Tm + i;
+  for (int j = lane; j < Tn; j += 32) {
+    const float p = row[j] / ssum;
+    row[j] = p;
+    rq[j] = mass_of(p);
+    if (out.pbar) out.pbar[rowid * Tn + j] = p;
+  }
+  __syncwarp();
+  select_row_warp(reinterpret_cast<const uint32_t*>(row), rq, Tn, K, thr, out.row_cnt + rowid,
+                  out.row_idx + rowid * Tn, bits + rowid * W, out.bitmap ? out.bitmap + rowid * Tn : nullptr,
+                  status);
 }
 
 // selection alone on a given P-bar: one warp per row, 8 rows per CTA
 __global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ pbar, int Tm, int Tn, int K,
-                                                     unsigned long long thr, MaskOut out,
-                                                     uint32_t* __restrict__ bits, int W, int* status) {
+                                                     double thr, MaskOut out, uint32_t* __restrict__ bits, int W,
+                                                     int* status) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  WarpHist* hist = reinterpret_cast<WarpHist*>(smem_raw);   // [8]
-  float* rows = reinterpret_cast<float*>(hist + 8);          // [8][Tn]
   const int w = threadIdx.x >> 5;
+  double* rq = reinterpret_cast<double*>(smem_raw) + (size_t)w * Tn;           // [8][Tn]
+  uint32_t* keys = reinterpret_cast<uint32_t*>(reinterpret_cast<double*>(smem_raw) + (size_t)8 * Tn) +
+                   (size_t)w * Tn;                                              // [8][Tn]
   const uint32_t lane = lane_id();
   const long long bh = blockIdx.y;
   const int i = blockIdx.x * 8 + w;
   if (i >= Tm) return;
   const long long rowid = bh * Tm + i;
-  float* row = rows + (long long)w * Tn;
-  for (int j = lane; j < Tn; j += 32) row[j] = pbar[rowid * Tn + j];
+  for (int j = lane; j < Tn; j += 32) {
+    const float p = pbar[rowid * Tn + j];
+    keys[j] = __float_as_uint(p);
+    rq[j] = mass_of(p);
+  }
   __syncwarp();
-  select_row_warp(row, Tn, K, thr, hist + w, out.row_cnt + rowid, out.row_idx + rowid * Tn, bits + rowid * W,
+  select_row_warp(keys, rq, Tn, K, thr, out.row_cnt + rowid, out.row_idx + rowid * Tn, bits + rowid * W,
                   out.bitmap ? out.bitmap + rowid * Tn : nullptr, status);
 }
 
@@ -398,44 +355,40 @@ cudaError_t launch_pool(const void* q, const void* k, float* qbar, float* kbar, 
 }
 
 static size_t pbar_select_smem(int d, int rows, int Tn) {
-  return (size_t)rows * d * 4 + ((size_t)rows * Tn + 1) * 4 + 8 * sizeof(WarpHist) + 16;
+  return (size_t)rows * Tn * 8 + (size_t)rows * d * 4 + (size_t)rows * Tn * 4;
 }
 
 template <int D, int ROWS>
 static cudaError_t launch_pbar_select_t(const float* qbar, const float* kbar, int BH, int Tm, int Tn, int K,
-                                        unsigned long long thr, const MaskOut& out, uint32_t* bits, int W,
-                                        int* status, cudaStream_t s) {
+                                        double thr, const MaskOut& out, uint32_t* bits, int W, int* status,
+                                        cudaStream_t s) {
   const size_t smem = pbar_select_smem(D, ROWS, Tn);
   cudaError_t e = cudaFuncSetAttribute(pbar_select_kernel<D, ROWS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((Tm + ROWS - 1) / ROWS, BH);
-  pbar_select_kernel<D, ROWS><<<grid, 256, smem, s>>>(qbar, kbar, Tm, Tn, 1.0f / sqrtf((float)D), K, thr, out, bits,
-                                                      W, status);
+  pbar_select_kernel<D, ROWS><<<grid, ROWS * 32, smem, s>>>(qbar, kbar, Tm, Tn, 1.0f / sqrtf((float)D), K, thr, out,
+                                                            bits, W, status);
   return cudaGetLastError();
 }
 
 cudaError_t launch_pbar_select(const float* qbar, const float* kbar, int BH, int d, int Tm, int Tn, int K,
                                unsigned long long thr, const MaskOut& out, uint32_t* bits, int W, int* status,
                                cudaStream_t s) {
-  // 8 rows per CTA when few rows exist (fill the 148 SMs), else 16 (fewer Kbar re-reads)
-  const bool small = (long long)BH * Tm < 148LL * 16;
-  if (d == 128)
-    return small ? launch_pbar_select_t<128, 8>(qbar, kbar, BH, Tm, Tn, K, thr, out, bits, W, status, s)
-                 : launch_pbar_select_t<128, 16>(qbar, kbar, BH, Tm, Tn, K, thr, out, bits, W, status, s);
-  return small ? launch_pbar_select_t<64, 8>(qbar, kbar, BH, Tm, Tn, K, thr, out, bits, W, status, s)
-               : launch_pbar_select_t<64, 16>(qbar, kbar, BH, Tm, Tn, K, thr, out, bits, W, status, s);
+  const double thr_d = (double)thr;  // exact: thr <= 2^32
+  if (d == 128) return launch_pbar_select_t<128, 8>(qbar, kbar, BH, Tm, Tn, K, thr_d, out, bits, W, status, s);
+  return launch_pbar_select_t<64, 8>(qbar, kbar, BH, Tm, Tn, K, thr_d, out, bits, W, status, s);
 }
 
-size_t pbar_select_max_smem(int d, int Tn) { return pbar_select_smem(d, 16, Tn); }
+size_t pbar_select_max_smem(int d, int Tn) { return pbar_select_smem(d, 8, Tn); }
 
 cudaError_t launch_select(const float* pbar, int BH, int Tm, int Tn, int K, unsigned long long thr,
                           const MaskOut& out, uint32_t* bits, int W, int* status, cudaStream_t s) {
-  const size_t smem = 8 * sizeof(WarpHist) + (size_t)8 * Tn * 4;
+  const size_t smem = (size_t)8 * Tn * 12;
   cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((Tm + 7) / 8, BH);
-  select_kernel<<<grid, 256, smem, s>>>(pbar, Tm, Tn, K, thr, out, bits, W, status);
+  select_kernel<<<grid, 256, smem, s>>>(pbar, Tm, Tn, K, (double)thr, out, bits, W, status);
   return cudaGetLastError();
 }
 
