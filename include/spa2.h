@@ -132,7 +132,7 @@ SPA2_API spa2_status spa2_block_mask(const void* q, const void* k, int B, int H,
 /*
  * Step 3 alone on a caller-given P-bar (parity checks of the selection rule,
  * and masks computed elsewhere). Same rule and outputs as spa2_block_mask;
- * out->pbar is ignored. pbar entries must be finite and in [0, 1].
+ * out->pbar is ignored. pbar entries must be finite and in [0, 1]; T_n <= 2048.
  *   pbar : [B, H, T_m, T_n] fp32 device pointer
  *   ws   : spa2_workspace_bytes(SPA2_OP_SELECT, B, H, T_m, T_n, 0, 0) bytes
  */

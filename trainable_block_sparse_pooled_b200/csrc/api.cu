@@ -209,11 +209,9 @@ spa2_status spa2_block_mask(const void* q, const void* k, int B, int H, int N, i
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 
   SPA2_CUDA_TRY(cudaMemsetAsync(w.status, 0, 4, st));
-  SPA2_CUDA_TRY(launch_pool(q, k, w.qbar, w.kbar, (int)s.BH, s.N, s.d, s.Tm, s.Tn, bq, bkv, st));
   MaskOut mo{out->row_cnt, out->row_idx, out->pbar, out->bitmap};
-  SPA2_CUDA_TRY(launch_pbar_select(w.qbar, w.kbar, (int)s.BH, s.d, s.Tm, s.Tn, topk_count(k_frac, s.Tn),
-                                   topp_threshold(p_frac), mo, w.bits, s.W, w.status, st));
-  if (out->col_cnt) SPA2_CUDA_TRY(launch_csc(w.bits, (int)s.BH, s.Tm, s.Tn, s.W, out->col_cnt, out->col_idx, st));
+  SPA2_CUDA_TRY(launch_mask(q, k, w.qbar, w.kbar, (int)s.BH, s.N, s.d, s.Tm, s.Tn, bq, bkv, topk_count(k_frac, s.Tn),
+                            topp_threshold(p_frac), mo, out->col_cnt, out->col_idx, w.bits, s.W, w.status, st));
   return SPA2_OK;
 }
 
@@ -222,7 +220,7 @@ spa2_status spa2_select_blocks(const float* pbar, int B, int H, int Tm, int Tn, 
   if (!pbar || !out || !out->row_cnt || !out->row_idx) return SPA2_ERR_INVALID_ARG;
   if ((out->col_cnt == nullptr) != (out->col_idx == nullptr)) return SPA2_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || Tm < 1 || Tn < 1) return SPA2_ERR_INVALID_ARG;
-  if (Tn > 4096 || Tm > 65535 || (long long)B * H > 65535) return SPA2_ERR_UNSUPPORTED;
+  if (Tn > 2048 || Tm > 65535 || (long long)B * H > 65535) return SPA2_ERR_UNSUPPORTED;
   if (!frac_ok(k_frac) || !frac_ok(p_frac)) return SPA2_ERR_UNSUPPORTED;
   if (!ws || !aligned(ws, 256)) return SPA2_ERR_WORKSPACE;
   const size_t need = spa2_workspace_bytes(SPA2_OP_SELECT, B, H, Tm, Tn, 0, 0);

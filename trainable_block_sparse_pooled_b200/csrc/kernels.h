@@ -15,12 +15,9 @@ struct MaskOut {
 };
 
 // mask.cu
-cudaError_t launch_pool(const void* q, const void* k, float* qbar, float* kbar, int BH, int N, int d, int Tm, int Tn,
-                        int bq, int bkv, cudaStream_t s);
-cudaError_t launch_pbar_select(const float* qbar, const float* kbar, int BH, int d, int Tm, int Tn, int K,
-                               unsigned long long thr, const MaskOut& out, uint32_t* bits, int W, int* status,
-                               cudaStream_t s);
-size_t pbar_select_max_smem(int d, int Tn);
+cudaError_t launch_mask(const void* q, const void* k, float* qbar, float* kbar, int BH, int N, int d, int Tm, int Tn,
+                        int bq, int bkv, int K, unsigned long long thr, const MaskOut& out, int* col_cnt,
+                        int* col_idx, uint32_t* bits, int W, int* status, cudaStream_t s);
 cudaError_t launch_select(const float* pbar, int BH, int Tm, int Tn, int K, unsigned long long thr,
                           const MaskOut& out, uint32_t* bits, int W, int* status, cudaStream_t s);
 cudaError_t launch_csc(const uint32_t* bits, int BH, int Tm, int Tn, int W, int* col_cnt, int* col_idx,
