@@ -211,7 +211,8 @@ spa2_status spa2_block_mask(const void* q, const void* k, int B, int H, int N, i
   SPA2_CUDA_TRY(cudaMemsetAsync(w.status, 0, 4, st));
   MaskOut mo{out->row_cnt, out->row_idx, out->pbar, out->bitmap};
   SPA2_CUDA_TRY(launch_mask(q, k, w.qbar, w.kbar, (int)s.BH, s.N, s.d, s.Tm, s.Tn, bq, bkv, topk_count(k_frac, s.Tn),
-                            topp_threshold(p_frac), mo, out->col_cnt, out->col_idx, w.bits, s.W, w.status, st));
+                            topp_threshold(p_frac), mo, out->col_cnt, out->col_idx, w.bits, s.W, w.status,
+                            g_wait_limit_ns, st));
   return SPA2_OK;
 }
 

@@ -93,14 +93,22 @@ struct WaitCtx {
 
 SPA2_DEV bool wait_bar(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
+  // try_wait suspends the thread for a while when the phase is open, so polling it
+  // is cheap; the abort flag and the clock (a special-register read that would
+  // compete with exp2 for issue) are looked at only every 64 polls
+  uint64_t t0 = 0;
+  for (uint32_t n = 1;; ++n) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (*w.abort_flag) return false;
-    if (globaltimer_ns() - t0 > w.limit_ns) {
-      report(w.status, SPA2_ERR_DEVICE_TIMEOUT);
-      *w.abort_flag = 1;
-      return false;
+    if ((n & 63u) == 0u) {
+      if (*w.abort_flag) return false;
+      const uint64_t t = globaltimer_ns();
+      if (t0 == 0) {
+        t0 = t;
+      } else if (t - t0 > w.limit_ns) {
+        report(w.status, SPA2_ERR_DEVICE_TIMEOUT);
+        *w.abort_flag = 1;
+        return false;
+      }
     }
   }
 }
@@ -117,6 +125,15 @@ SPA2_DEV void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int 
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+// untiled bulk copy global -> shared (16-byte aligned addresses, size multiple of 16)
+SPA2_DEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
 

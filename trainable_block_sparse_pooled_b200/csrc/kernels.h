@@ -17,7 +17,8 @@ struct MaskOut {
 // mask.cu
 cudaError_t launch_mask(const void* q, const void* k, float* qbar, float* kbar, int BH, int N, int d, int Tm, int Tn,
                         int bq, int bkv, int K, unsigned long long thr, const MaskOut& out, int* col_cnt,
-                        int* col_idx, uint32_t* bits, int W, int* status, cudaStream_t s);
+                        int* col_idx, uint32_t* bits, int W, int* status, unsigned long long wait_limit_ns,
+                        cudaStream_t s);
 cudaError_t launch_select(const float* pbar, int BH, int Tm, int Tn, int K, unsigned long long thr,
                           const MaskOut& out, uint32_t* bits, int W, int* status, cudaStream_t s);
 cudaError_t launch_csc(const uint32_t* bits, int BH, int Tm, int Tn, int W, int* col_cnt, int* col_idx,

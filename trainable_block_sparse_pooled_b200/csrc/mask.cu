@@ -4,13 +4,10 @@
 //   pool_kernel    one CTA per block: mean of each q-block (b_q rows) and kv-block
 //                  (b_kv rows) of Q / K -> Qbar [B,H,Tm,d], Kbar [B,H,Tn,d] fp32.
 //   select_kernel  8 q-block rows of one head per CTA, one warp per row: fp32
-//                  logits against Kbar (staged through smem with cp.async), softmax
-//                  -> P-bar, hybrid selection -> CSR, kept-bit words, optional
-//                  P-bar / uint8 bitmap. Launched as a programmatic dependent of
-//                  pool_kernel (its launch overlaps the pool's tail; it waits for
-//                  the pool's results with griddepcontrol.wait).
-//   csc_kernel     kept-bit words -> CSC, one warp per kv-block column (dependent
-//                  launch after select_kernel).
+//                  logits against Kbar (streamed through a 4-deep smem ring with
+//                  bulk async copies), softmax -> P-bar, hybrid selection -> CSR,
+//                  kept-bit words, optional P-bar / uint8 bitmap.
+//   csc_kernel     kept-bit words -> CSC, one warp per kv-block column.
 //   pbar_select_kernel  the selection alone on a caller-given P-bar.
 //
 // Selection is exact integer work on the float32 P-bar: ranks are (value desc,
@@ -37,10 +34,6 @@ constexpr int KCH = 32;  // Kbar rows per staged chunk
 SPA2_DEV unsigned long long mass_of(float p) {
   return __float2ull_rz(p * 4294967296.0f);  // exact: power-of-two scale of p in [0, 1]
 }
-
-// griddepcontrol: let a dependent launch start / wait for the grid this one depends on
-SPA2_DEV void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-SPA2_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------
 // pooling of one block: 16-byte streaming loads, all rows of a thread in flight
@@ -204,13 +197,23 @@ SPA2_DEV void csc_column_warp(const uint32_t* __restrict__ head_bits, int Tm, in
                               int* col_idx_out) {
   const uint32_t lane = lane_id();
   const uint32_t lt = (1u << lane) - 1u;
+  const uint32_t* col = head_bits + (c >> 5);
   int running = 0;
-  for (int base = 0; base < Tm; base += 32) {
-    const int i = base + (int)lane;
-    const bool bit = (i < Tm) && ((head_bits[(long long)i * W + (c >> 5)] >> (c & 31)) & 1u);
-    const uint32_t bal = __ballot_sync(0xffffffff, bit);
-    if (bit) col_idx_out[running + __popc(bal & lt)] = i;
-    running += __popc(bal);
+  for (int base = 0; base < Tm; base += 32 * 8) {
+    uint32_t w8[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {  // all loads of 8 row groups in flight
+      const int i = base + 32 * u + (int)lane;
+      w8[u] = (i < Tm) ? col[(long long)i * W] : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = base + 32 * u + (int)lane;
+      const bool bit = (w8[u] >> (c & 31)) & 1u;
+      const uint32_t bal = __ballot_sync(0xffffffff, bit);
+      if (bit) col_idx_out[running + __popc(bal & lt)] = i;
+      running += __popc(bal);
+    }
   }
   if (lane == 0) *col_cnt_out = running;
 }
@@ -220,11 +223,11 @@ SPA2_DEV void csc_column_warp(const uint32_t* __restrict__ head_bits, int Tm, in
 template <int D>
 __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ q,
                                                    const __nv_bfloat16* __restrict__ k, float* __restrict__ qbar,
-                                                   float* __restrict__ kbar, int N, int Tm, int Tn, int bq, int bkv) {
+                                                   float* __restrict__ kbar, int h0, int N, int Tm, int Tn, int bq,
+                                                   int bkv) {
   __shared__ float red[(256 / (D / 8)) * (D + 1)];
-  pdl_trigger();
   const int blk = blockIdx.x;
-  const long long h = blockIdx.y;
+  const long long h = h0 + blockIdx.y;
   const __nv_bfloat16* src;
   float* dst;
   int rows;
@@ -241,64 +244,89 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
   pool_block<D>(src, rows, dst, red);
 }
 
-// 8 rows (one per warp) of head blockIdx.y: logits, softmax, selection
+// 8 rows (one per warp) of head h0 + blockIdx.y: logits, softmax, selection
 template <int D, int E>
-__global__ void __launch_bounds__(256) select_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
-                                                     int Tm, int Tn, int W, float inv_sqrt_d, int K,
-                                                     unsigned long long thr, MaskOut out,
-                                                     uint32_t* __restrict__ bits, int* status) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  float* qb = reinterpret_cast<float*>(smem_raw);  // [ROWS][D]
-  float* kst = qb + ROWS * D;                      // [2][KCH][D+4]
-  float* lrows = kst + 2 * KCH * (D + 4);          // [ROWS][32 E]
-  pdl_trigger();
-  pdl_wait();  // Qbar / Kbar of pool_kernel
+__global__ void __launch_bounds__(256, (E <= 16 ? 2 : 1)) select_kernel(const float* __restrict__ qbar,
+                                                        const float* __restrict__ kbar, int h0, int Tm, int Tn, int W,
+                                                        float inv_sqrt_d, int K, unsigned long long thr, MaskOut out,
+                                                        uint32_t* __restrict__ bits, int* status,
+                                                        unsigned long long wait_limit_ns) {
+  constexpr int NST = 4;                                   // ring depth
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  float* ring = reinterpret_cast<float*>(smem_raw);        // [NST][KCH][D], unpadded
+  float* qb = ring + NST * KCH * D;                        // [ROWS][D]
+  float* lrows = qb + ROWS * D;                            // [ROWS][32 E]
+  uint64_t* full = reinterpret_cast<uint64_t*>(lrows + ROWS * 32 * E);  // [NST]
+  __shared__ int abort_flag;
   const int warp = threadIdx.x >> 5;
   const uint32_t lane = lane_id();
-  const long long h = blockIdx.y;
+  const long long h = h0 + blockIdx.y;
   const int i0 = blockIdx.x * ROWS;
   const float* kb = kbar + h * Tn * D;
+  const int nch = (Tn + KCH - 1) / KCH;
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < NST; ++st) mbar_init(&full[st], 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const WaitCtx wc{&abort_flag, status, wait_limit_ns};
+  int issued = 0;  // meaningful in thread 0 only
+  auto issue = [&](int ch) {  // thread 0 only
+    const int rows = min(KCH, Tn - ch * KCH);
+    const uint32_t bytes = (uint32_t)rows * D * 4;
+    uint64_t* bar = &full[ch % NST];
+    mbar_expect_tx(bar, bytes);
+    bulk_load(ring + (ch % NST) * KCH * D, kb + (long long)ch * KCH * D, bytes, bar);
+    issued = ch + 1;
+  };
+  if (threadIdx.x == 0)
+    for (int ch = 0; ch < min(NST - 1, nch); ++ch) issue(ch);
   for (int e = threadIdx.x; e < ROWS * D; e += 256) {
     const int rr = e / D;
     qb[e] = (i0 + rr < Tm) ? qbar[(h * Tm + i0 + rr) * D + (e % D)] : 0.f;
   }
-  const int nch = (Tn + KCH - 1) / KCH;
-  auto stage = [&](int ch, int buf) {
-    float* dstb = kst + buf * KCH * (D + 4);
-    for (int e = threadIdx.x; e < KCH * (D / 4); e += 256) {
-      const int rr = e / (D / 4), c4 = e % (D / 4);
-      const int row = ch * KCH + rr;
-      const bool ok = row < Tn;
-      cp_async16(dstb + rr * (D + 4) + c4 * 4, kb + (long long)(ok ? row : 0) * D + c4 * 4, ok ? 16u : 0u);
-    }
-    cp_async_commit();
-  };
-  stage(0, 0);
+  __syncthreads();
   float* lrow = lrows + warp * 32 * E;
-  for (int ch = 0; ch < nch; ++ch) {
-    if (ch + 1 < nch) {
-      stage(ch + 1, (ch + 1) & 1);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
+  const float4* qr = reinterpret_cast<const float4*>(qb + warp * D);
+  bool ok = true;
+  int ch = 0;
+  for (; ch < nch; ++ch) {
+    if (threadIdx.x == 0 && ch + NST - 1 < nch) issue(ch + NST - 1);  // its slot was freed last iteration
+    ok = wait_bar(&full[ch % NST], (ch / NST) & 1, wc);
+    if (__syncthreads_or(!ok)) {
+      ok = false;
+      break;
     }
-    __syncthreads();
-    // lane l: logit of row (i0 + warp) against Kbar row ch*KCH + l, sequential over d
-    const float4* kr = reinterpret_cast<const float4*>(kst + (ch & 1) * KCH * (D + 4) + lane * (D + 4));
-    const float4* qr = reinterpret_cast<const float4*>(qb + warp * D);
-    float acc = 0.f;
-#pragma unroll 8
-    for (int e = 0; e < D / 4; ++e) {
-      const float4 kv = kr[e];
-      const float4 qv = qr[e];
-      acc = fmaf(qv.x, kv.x, acc);
-      acc = fmaf(qv.y, kv.y, acc);
-      acc = fmaf(qv.z, kv.z, acc);
-      acc = fmaf(qv.w, kv.w, acc);
-    }
+    // lane l: logit of row (i0 + warp) against Kbar row ch*KCH + l; each lane walks
+    // d in its own rotated order (conflict-free 16-byte smem reads), sequentially
     const int c = ch * KCH + (int)lane;
-    if (c < Tn) lrow[c] = acc * inv_sqrt_d;
-    __syncthreads();  // the buffer is refilled next iteration
+    if (c < Tn) {
+      const float4* kr = reinterpret_cast<const float4*>(ring + (ch % NST) * KCH * D + lane * D);
+      float acc = 0.f;
+#pragma unroll 8
+      for (int t = 0; t < D / 4; ++t) {
+        const int e = (t + (int)lane) & (D / 4 - 1);
+        const float4 kv = kr[e];
+        const float4 qv = qr[e];
+        acc = fmaf(qv.x, kv.x, acc);
+        acc = fmaf(qv.y, kv.y, acc);
+        acc = fmaf(qv.z, kv.z, acc);
+        acc = fmaf(qv.w, kv.w, acc);
+      }
+      lrow[c] = acc * inv_sqrt_d;
+    }
+    __syncthreads();  // every warp is done with this slot
+  }
+  if (!ok) {
+    // never leave with bulk copies in flight: wait (bounded) for the issued ones
+    if (threadIdx.x == 0) {
+      __shared__ int never;
+      never = 0;
+      const WaitCtx dw{&never, nullptr, wait_limit_ns};
+      for (int c2 = ch; c2 < issued; ++c2) wait_bar(&full[c2 % NST], (c2 / NST) & 1, dw);
+    }
+    return;
   }
   const int i = i0 + warp;
   if (i >= Tm) return;
@@ -340,10 +368,9 @@ __global__ void __launch_bounds__(256) pbar_select_kernel(const float* __restric
 }
 
 // kept-bit words [B*H, Tm, W] -> CSC; one warp per kv-block column, 8 per CTA
-__global__ void __launch_bounds__(256) csc_kernel(const uint32_t* __restrict__ bits, int Tm, int Tn, int W,
-                                                  int* __restrict__ col_cnt, int* __restrict__ col_idx) {
-  pdl_wait();  // kept-bit words of the selection kernel (no-op without a dependent launch)
-  const long long bh = blockIdx.y;
+__global__ void __launch_bounds__(256) csc_kernel(const uint32_t* __restrict__ bits, int h0, int Tm, int Tn,
+                                                  int W, int* __restrict__ col_cnt, int* __restrict__ col_idx) {
+  const long long bh = h0 + blockIdx.y;
   const int c = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (c >= Tn) return;
   csc_column_warp(bits + bh * Tm * W, Tm, W, c, col_cnt + bh * Tn + c, col_idx + (bh * Tn + c) * Tm);
@@ -352,62 +379,49 @@ __global__ void __launch_bounds__(256) csc_kernel(const uint32_t* __restrict__ b
 // ---------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------
-template <typename... KArgs, typename... Args>
-static cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                                    Args... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
-}
-
 template <int D, int E>
-static cudaError_t launch_select_t(const float* qbar, const float* kbar, int BH, int Tm, int Tn, int W, int K,
+static cudaError_t launch_select_t(const float* qbar, const float* kbar, int h0, int nh, int Tm, int Tn, int W, int K,
                                    unsigned long long thr, const MaskOut& out, uint32_t* bits, int* status,
-                                   cudaStream_t s) {
-  const size_t smem = ((size_t)ROWS * D + (size_t)2 * KCH * (D + 4) + (size_t)ROWS * 32 * E) * 4;
+                                   unsigned long long wait_limit_ns, cudaStream_t s) {
+  const size_t smem = ((size_t)4 * KCH * D + (size_t)ROWS * D + (size_t)ROWS * 32 * E) * 4 + 4 * 8;
   cudaError_t e = cudaFuncSetAttribute(select_kernel<D, E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_dependent(select_kernel<D, E>, dim3((Tm + ROWS - 1) / ROWS, BH), dim3(256), smem, s, qbar, kbar, Tm,
-                          Tn, W, 1.0f / sqrtf((float)D), K, thr, out, bits, status);
+  select_kernel<D, E><<<dim3((Tm + ROWS - 1) / ROWS, nh), 256, smem, s>>>(
+      qbar, kbar, h0, Tm, Tn, W, 1.0f / sqrtf((float)D), K, thr, out, bits, status, wait_limit_ns);
+  return cudaGetLastError();
 }
 
 template <int D>
-static cudaError_t launch_select_d(const float* qbar, const float* kbar, int BH, int Tm, int Tn, int W, int K,
+static cudaError_t launch_select_d(const float* qbar, const float* kbar, int h0, int nh, int Tm, int Tn, int W, int K,
                                    unsigned long long thr, const MaskOut& out, uint32_t* bits, int* status,
-                                   cudaStream_t s) {
+                                   unsigned long long wl, cudaStream_t s) {
   const int e = (Tn + 31) / 32;
-  if (e <= 8) return launch_select_t<D, 8>(qbar, kbar, BH, Tm, Tn, W, K, thr, out, bits, status, s);
-  if (e <= 16) return launch_select_t<D, 16>(qbar, kbar, BH, Tm, Tn, W, K, thr, out, bits, status, s);
-  if (e <= 40) return launch_select_t<D, 40>(qbar, kbar, BH, Tm, Tn, W, K, thr, out, bits, status, s);
-  return launch_select_t<D, 64>(qbar, kbar, BH, Tm, Tn, W, K, thr, out, bits, status, s);
+  if (e <= 8) return launch_select_t<D, 8>(qbar, kbar, h0, nh, Tm, Tn, W, K, thr, out, bits, status, wl, s);
+  if (e <= 16) return launch_select_t<D, 16>(qbar, kbar, h0, nh, Tm, Tn, W, K, thr, out, bits, status, wl, s);
+  if (e <= 40) return launch_select_t<D, 40>(qbar, kbar, h0, nh, Tm, Tn, W, K, thr, out, bits, status, wl, s);
+  return launch_select_t<D, 64>(qbar, kbar, h0, nh, Tm, Tn, W, K, thr, out, bits, status, wl, s);
 }
 
 cudaError_t launch_mask(const void* q, const void* k, float* qbar, float* kbar, int BH, int N, int d, int Tm, int Tn,
                         int bq, int bkv, int K, unsigned long long thr, const MaskOut& out, int* col_cnt,
-                        int* col_idx, uint32_t* bits, int W, int* status, cudaStream_t s) {
+                        int* col_idx, uint32_t* bits, int W, int* status, unsigned long long wait_limit_ns,
+                        cudaStream_t s) {
   dim3 grid(Tm + Tn, BH);
   if (d == 128)
-    pool_kernel<128><<<grid, 256, 0, s>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qbar, kbar, N, Tm, Tn,
+    pool_kernel<128><<<grid, 256, 0, s>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qbar, kbar, 0, N, Tm, Tn,
                                           bq, bkv);
   else
-    pool_kernel<64><<<grid, 256, 0, s>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qbar, kbar, N, Tm, Tn,
+    pool_kernel<64><<<grid, 256, 0, s>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qbar, kbar, 0, N, Tm, Tn,
                                          bq, bkv);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  e = (d == 128) ? launch_select_d<128>(qbar, kbar, BH, Tm, Tn, W, K, thr, out, bits, status, s)
-                 : launch_select_d<64>(qbar, kbar, BH, Tm, Tn, W, K, thr, out, bits, status, s);
+  e = (d == 128) ? launch_select_d<128>(qbar, kbar, 0, BH, Tm, Tn, W, K, thr, out, bits, status, wait_limit_ns, s)
+                 : launch_select_d<64>(qbar, kbar, 0, BH, Tm, Tn, W, K, thr, out, bits, status, wait_limit_ns, s);
   if (e != cudaSuccess) return e;
-  if (col_cnt)
-    e = launch_dependent(csc_kernel, dim3((Tn + 7) / 8, BH), dim3(256), 0, s, (const uint32_t*)bits, Tm, Tn, W,
-                         col_cnt, col_idx);
+  if (col_cnt) {
+    csc_kernel<<<dim3((Tn + 7) / 8, BH), 256, 0, s>>>(bits, 0, Tm, Tn, W, col_cnt, col_idx);
+    e = cudaGetLastError();
+  }
   return e;
 }
 
@@ -429,7 +443,7 @@ cudaError_t launch_select(const float* pbar, int BH, int Tm, int Tn, int K, unsi
 cudaError_t launch_csc(const uint32_t* bits, int BH, int Tm, int Tn, int W, int* col_cnt, int* col_idx,
                        cudaStream_t s) {
   dim3 grid((Tn + 7) / 8, BH);
-  csc_kernel<<<grid, 256, 0, s>>>(bits, Tm, Tn, W, col_cnt, col_idx);
+  csc_kernel<<<grid, 256, 0, s>>>(bits, 0, Tm, Tn, W, col_cnt, col_idx);
   return cudaGetLastError();
 }
 
