@@ -130,6 +130,34 @@ SPA2_API spa2_status spa2_block_mask(const void* q, const void* k, int B, int H,
                             spa2_stream_t stream);
 
 /*
+ * spa2_block_mask without a caller workspace. The method has no counterpart
+ * of this entry point: it exists for callers that cannot hand the library a
+ * workspace at call time, such as a plain C host program on a fixed memory
+ * plan with no device allocator of its own, or a step loop that must not call
+ * cudaMalloc (which synchronises the whole device) between kernels.
+ * Computes exactly what spa2_block_mask computes, with the same kernels.
+ *   scratch: one file-scope device array of SPA2_NOALLOC_MASK_SCRATCH_BYTES
+ *            per device, part of the library's image; nothing is allocated
+ *            by the call. A shape whose mask workspace
+ *            (spa2_workspace_bytes(SPA2_OP_MASK, ...)) exceeds that size is
+ *            refused with SPA2_ERR_WORKSPACE before any launch.
+ *   setup:   the first call on a device (with that device current) looks the
+ *            array's address up once and caches it; make that first call
+ *            before any stream capture begins on that device.
+ *   status:  NULL, or a 4-byte-aligned device int the caller owns; the call
+ *            copies the device-side status word there (stream-ordered). Read
+ *            it with spa2_stream_status(status, stream).
+ *   races:   all calls on one device share the array. Calls issued one after
+ *            another on one stream are safe; calls whose executions overlap
+ *            (other streams, other host threads) race and give wrong masks.
+ * Arguments and outputs otherwise as spa2_block_mask.
+ */
+#define SPA2_NOALLOC_MASK_SCRATCH_BYTES (64u << 20) /* 64 MiB */
+SPA2_API spa2_status spa2_block_mask_noalloc(const void* q, const void* k, int B, int H, int N, int d, int bq,
+                                    int bkv, float k_frac, float p_frac, const spa2_mask* out, int* status,
+                                    spa2_stream_t stream);
+
+/*
  * Step 3 alone on a caller-given P-bar (parity checks of the selection rule,
  * and masks computed elsewhere). Same rule and outputs as spa2_block_mask;
  * out->pbar is ignored. pbar entries must be finite and in [0, 1]; T_n <= 2048.

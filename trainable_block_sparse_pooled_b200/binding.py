@@ -53,6 +53,9 @@ _SIGS = {
     "spa2_block_mask": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int] * 6
                         + [ctypes.c_float, ctypes.c_float, ctypes.POINTER(spa2_mask), ctypes.c_void_p,
                            ctypes.c_size_t, ctypes.c_void_p]),
+    "spa2_block_mask_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int] * 6
+                                + [ctypes.c_float, ctypes.c_float, ctypes.POINTER(spa2_mask), ctypes.c_void_p,
+                                   ctypes.c_void_p]),
     "spa2_select_blocks": (ctypes.c_int, [ctypes.c_void_p] + [ctypes.c_int] * 4
                            + [ctypes.c_float, ctypes.c_float, ctypes.POINTER(spa2_mask), ctypes.c_void_p,
                               ctypes.c_size_t, ctypes.c_void_p]),
@@ -112,6 +115,11 @@ def spa2_workspace_bytes(op, B, H, N, d, bq=BQ, bkv=BKV) -> int:
 def spa2_block_mask(q, k, B, H, N, d, bq, bkv, k_frac, p_frac, mask: spa2_mask, ws, ws_bytes, stream) -> int:
     return lib().spa2_block_mask(q, k, B, H, N, d, bq, bkv, k_frac, p_frac, ctypes.byref(mask), ws, ws_bytes,
                                  stream)
+
+
+def spa2_block_mask_noalloc(q, k, B, H, N, d, bq, bkv, k_frac, p_frac, mask: spa2_mask, status, stream) -> int:
+    return lib().spa2_block_mask_noalloc(q, k, B, H, N, d, bq, bkv, k_frac, p_frac, ctypes.byref(mask), status,
+                                         stream)
 
 
 def spa2_select_blocks(pbar, B, H, Tm, Tn, k_frac, p_frac, mask: spa2_mask, ws, ws_bytes, stream) -> int:
