@@ -185,6 +185,8 @@ __global__ void __launch_bounds__(192, 2) fwd_kernel(const __grid_constant__ CUt
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
     float m_use = -INFINITY, l = 0.f;
     bool ok = n > 0;
+    // only the kv-block Tn-1 is ragged, and the ascending list holds it last
+    const int last_valid = (n > 0 && kv_list[n - 1] == Tn - 1) ? (N - (Tn - 1) * 64) : 64;
     for (int t = 0; t < n && ok; ++t) {
       const int s = t & 1;
       if (!wait_warp(&sm.s_full[s], (t >> 1) & 1, wc)) {
@@ -192,24 +194,23 @@ __global__ void __launch_bounds__(192, 2) fwd_kernel(const __grid_constant__ CUt
         break;
       }
       tc_fence_after();
-      const int j = kv_list[t];
-      const int valid = (j == Tn - 1) ? (N - j * 64) : 64;
-      uint32_t ra[32], rb[32];
-      tmem_ld32(tl + s * 64, ra);
-      tmem_ld32(tl + s * 64 + 32, rb);
+      const int valid = (t == n - 1) ? last_valid : 64;
+      uint32_t sv[64];
+      tmem_ld64(tl + s * 64, sv);
       tmem_wait_ld();
-      float mx = -INFINITY;
-      if (valid >= 64) {
+      if (valid < 64) {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) mx = fmaxf(mx, fmaxf(__uint_as_float(ra[c]), __uint_as_float(rb[c])));
-      } else {
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          if (c >= valid) ra[c] = __float_as_uint(-INFINITY);
-          if (c + 32 >= valid) rb[c] = __float_as_uint(-INFINITY);
-          mx = fmaxf(mx, fmaxf(__uint_as_float(ra[c]), __uint_as_float(rb[c])));
-        }
+        for (int c = 0; c < 64; ++c)
+          if (c >= valid) sv[c] = __float_as_uint(-INFINITY);
       }
+      // row max as a tree (independent partial maxima)
+      float m4[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) m4[q] = __uint_as_float(sv[q]);
+#pragma unroll
+      for (int c = 8; c < 64; ++c) m4[c & 7] = fmaxf(m4[c & 7], __uint_as_float(sv[c]));
+      const float mx = fmaxf(fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])),
+                             fmaxf(fmaxf(m4[4], m4[5]), fmaxf(m4[6], m4[7])));
       const float m_new = fmaxf(m_use, mx * scale_log2);
       float alpha = 1.f;
       bool rescale = false;
@@ -223,17 +224,15 @@ __global__ void __launch_bounds__(192, 2) fwd_kernel(const __grid_constant__ CUt
       }
       const float neg_m = -m_use;
       uint32_t pk[32];
-      float rs = 0.f;
+      float rsum[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const float p0 = fast_exp2(fmaf(__uint_as_float(ra[2 * c]), scale_log2, neg_m));
-        const float p1 = fast_exp2(fmaf(__uint_as_float(ra[2 * c + 1]), scale_log2, neg_m));
-        const float p2 = fast_exp2(fmaf(__uint_as_float(rb[2 * c]), scale_log2, neg_m));
-        const float p3 = fast_exp2(fmaf(__uint_as_float(rb[2 * c + 1]), scale_log2, neg_m));
-        rs += (p0 + p1) + (p2 + p3);
+      for (int c = 0; c < 32; ++c) {
+        const float p0 = fast_exp2(fmaf(__uint_as_float(sv[2 * c]), scale_log2, neg_m));
+        const float p1 = fast_exp2(fmaf(__uint_as_float(sv[2 * c + 1]), scale_log2, neg_m));
+        rsum[c & 3] += p0 + p1;
         pk[c] = pack_f16(p0, p1);
-        pk[16 + c] = pack_f16(p2, p3);
       }
+      const float rs = (rsum[0] + rsum[1]) + (rsum[2] + rsum[3]);
       l += rs;
       tmem_st32(tl + s * 64, pk);
       if (t >= 1 && !wait_warp(&sm.o_done, (t - 1) & 1, wc)) {
