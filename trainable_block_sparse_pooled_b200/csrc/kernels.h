@@ -45,18 +45,22 @@ cudaError_t launch_v_to_f16(const void* v, void* v16, long long elems, int* stat
 
 // attn_bwd.cu
 struct BwdArgs {
-  const CUtensorMap* tm_q;    // box {64, 128, 1}
-  const CUtensorMap* tm_k;    // box {64, 64, 1}
-  const CUtensorMap* tm_v;    // box {64, 64, 1}
-  const CUtensorMap* tm_do;   // box {64, 128, 1}
+  const CUtensorMap* tm_q;    // Q bf16, box {64, 128, 1}
+  const CUtensorMap* tm_k;    // K bf16, box {64, 64, 1}
+  const CUtensorMap* tm_v;    // fp16 copy of V, box {64, 64, 1}
+  const CUtensorMap* tm_do;   // fp16 copy of dO, box {64, 128, 1}
+  const CUtensorMap* tm_dq;   // fp32 dQ accumulator, box {32, 128, 1}
   const void* o;
   const void* o_lo;   // may be null
   const void* dout;
+  const void* v;
   const float* lse;
   const int* col_cnt;
   const int* col_idx;
   float* dvec;     // [BH, N]
   float* dq_acc;   // [BH, N, d]
+  void* do16;      // [BH, N, d] fp16
+  void* v16;       // [BH, N, d] fp16
   void* dq;
   void* dk;
   void* dv;
