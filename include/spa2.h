@@ -76,8 +76,8 @@ typedef enum {
  *   pbar    [B, H, T_m, T_n]  fp32   pooled attention P-bar, or NULL
  *   bitmap  [B, H, T_m, T_n]  uint8  1 = kept, or NULL
  * spa2_sparse_attn_fwd reads row_cnt/row_idx; spa2_sparse_attn_bwd reads
- * col_cnt/col_idx; the mask builders write all non-NULL fields (col_* may be
- * NULL when no backward pass will follow).
+ * both; the mask builders write all non-NULL fields (col_* may be NULL when no
+ * backward pass will follow).
  */
 typedef struct {
   int32_t* row_cnt;
@@ -198,19 +198,25 @@ SPA2_API spa2_status spa2_sparse_attn_fwd(const void* q, const void* k, const vo
  *   dS_ij = P_ij * (dP_ij - D_i),  dQ_i = sum_j dS_ij K_j * scale,
  *   dK_j = sum_i dS_ij^T Q_i * scale.
  * The mask is held constant (no gradient through pooling or selection).
- * Precision: P and dS enter the dV, dK and dQ tensor-core products as
- * hi + lo bf16 pairs (about 16 mantissa bits) with fp32 accumulation, and D
- * uses o + o_lo when o_lo is given, so the gradients carry fp32-level error
- * before their final store.
+ * Precision: P enters dV = P^T dO as fp16 (P in [0, 1], 11-bit significand)
+ * against an fp16 copy of dO; dP = dO V^T takes fp16 copies of dO and V; dS
+ * enters dK and dQ as a hi + lo pair of bf16 values (about 16 significant
+ * bits); S = Q K^T takes the bf16 inputs; accumulation is fp32 throughout and
+ * D uses o + o_lo when o_lo is given. dO or V of magnitude > 65504 is clamped
+ * for the fp16 copies and reported as SPA2_ERR_RANGE.
+ * dK and dV are accumulated per kv-block (CSC column), dQ per q-block (CSR
+ * row, recomputing S and dP), so no output is accumulated atomically and the
+ * results are deterministic.
  *   q, k, v, o, dout : [B, H, N, d] bf16 device pointers (read only); o, o_lo
  *                      and lse are the forward outputs for the same mask
  *   o_lo             : optional [B, H, N, d] bf16 residual of O (or NULL)
  *   lse              : [B, H, N] fp32 device pointer
- *   mask             : host pointer to a spa2_mask; col_cnt/col_idx are read
+ *   mask             : host pointer to a spa2_mask; row_cnt/row_idx and
+ *                      col_cnt/col_idx are read
  *   dq, dk, dv       : [B, H, N, d] device outputs of type grad_dtype
  *   grad_dtype       : SPA2_DTYPE_BF16 or SPA2_DTYPE_F32
  *   ws               : spa2_workspace_bytes(SPA2_OP_BWD, ...) bytes (holds D
- *                      and, for bf16 gradients, the fp32 dQ accumulator)
+ *                      and the fp16 copies of dO and V)
  */
 SPA2_API spa2_status spa2_sparse_attn_bwd(const void* q, const void* k, const void* v, const void* o,
                                           const void* o_lo, const float* lse, const void* dout, int B, int H, int N,

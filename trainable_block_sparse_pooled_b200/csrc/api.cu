@@ -70,7 +70,6 @@ static MaskWs mask_ws(void* ws, const Shape& s) {
 struct BwdWs {
   int* status;
   float* dvec;
-  float* dq_acc;
   void* do16;
   void* v16;
   size_t bytes;
@@ -82,8 +81,6 @@ static BwdWs bwd_ws(void* ws, const Shape& s) {
   w.status = reinterpret_cast<int*>(base);
   w.dvec = reinterpret_cast<float*>(base + off);
   off += al256((size_t)s.BH * s.N * 4);
-  w.dq_acc = reinterpret_cast<float*>(base + off);
-  off += al256((size_t)s.BH * s.N * s.d * 4);
   w.do16 = base + off;
   off += al256((size_t)s.BH * s.N * s.d * 2);
   w.v16 = base + off;
@@ -119,20 +116,6 @@ static bool make_map(CUtensorMap* m, const void* ptr, const Shape& s, int rows, 
   cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
-// [BH, N, d] fp32 as {d, N, BH}; box {32, rows, 1} (128-byte rows), 128-byte swizzle
-static bool make_map_f32(CUtensorMap* m, const void* ptr, const Shape& s, int rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)s.d, (cuuint64_t)s.N, (cuuint64_t)s.BH};
-  cuuint64_t strides[2] = {(cuuint64_t)s.d * 4, (cuuint64_t)s.N * s.d * 4};
-  cuuint32_t box[3] = {32, (cuuint32_t)rows, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -293,7 +276,8 @@ spa2_status spa2_sparse_attn_bwd(const void* q, const void* k, const void* v, co
                                  int grad_dtype, void* ws, size_t ws_bytes, spa2_stream_t stream) {
   Shape s;
   spa2_status err;
-  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !mask || !mask->col_cnt || !mask->col_idx)
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !mask || !mask->row_cnt || !mask->row_idx ||
+      !mask->col_cnt || !mask->col_idx)
     return SPA2_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(o_lo, 16) ||
       !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4))
@@ -307,13 +291,13 @@ spa2_status spa2_sparse_attn_bwd(const void* q, const void* k, const void* v, co
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)d);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const bool f32 = grad_dtype == SPA2_DTYPE_F32;
-  CUtensorMap tq, tk, tv, tdo, tdq;
+  CUtensorMap tq, tk, tv, tdo;
   if (!make_map(&tq, q, s, 128) || !make_map(&tk, k, s, 64) || !make_map(&tv, w.v16, s, 64, true) ||
-      !make_map(&tdo, w.do16, s, 128, true) || !make_map_f32(&tdq, f32 ? dq : w.dq_acc, s, 128))
+      !make_map(&tdo, w.do16, s, 128, true))
     return SPA2_ERR_CUDA;
   SPA2_CUDA_TRY(cudaMemsetAsync(w.status, 0, 4, st));
-  BwdArgs a{&tq, &tk, &tv, &tdo, &tdq, o, o_lo, dout, v, lse, mask->col_cnt, mask->col_idx, w.dvec, w.dq_acc,
-            w.do16, w.v16, dq, dk, dv, f32 ? 1 : 0, (int)s.BH, s.N, s.Tm, s.Tn, scale,
+  BwdArgs a{&tq, &tk, &tv, &tdo, o, o_lo, dout, v, lse, mask->row_cnt, mask->row_idx, mask->col_cnt,
+            mask->col_idx, w.dvec, w.do16, w.v16, dq, dk, dv, f32 ? 1 : 0, (int)s.BH, s.N, s.Tm, s.Tn, scale,
             scale * 1.4426950408889634f, w.status, g_wait_limit_ns};
   SPA2_CUDA_TRY(launch_bwd(a, d, st));
   return SPA2_OK;

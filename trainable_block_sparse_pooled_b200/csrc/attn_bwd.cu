@@ -5,33 +5,32 @@
 //   dV_j += P^T dO_i      dP = dO_i V_j^T      dS = P * (dP - D_i)
 //   dQ_i += dS K_j * sc   dK_j += dS^T Q_i * sc,  D_i = rowsum(dO_i * O_i).
 //
-// bwd_pre_kernel   D = rowsum(dO * (O + O_lo)) in fp32, zeroes the fp32 dQ, and
-//                  writes fp16 copies of dO and V (for the fp16 products below;
-//                  |x| > 65504 is clamped and reported as SPA2_ERR_RANGE).
-// bwd_kernel       one CTA per (kv-block j, head), looping over the q-blocks i
-//                  that keep j (CSC column of j). Every GEMM is an M=128 tcgen05
-//                  MMA with fp32 accumulation in TMEM:
+// bwd_pre_kernel   D = rowsum(dO * (O + O_lo)) in fp32, and fp16 copies of dO
+//                  and V for the fp16 products below (|x| > 65504 is clamped
+//                  and reported as SPA2_ERR_RANGE).
+// bwd_dkdv_kernel  one CTA per (kv-block j, head), looping over the q-blocks i
+//                  that keep j (CSC column of j), accumulating dV_j and dK_j in
+//                  TMEM (tcgen05 MMAs, fp32 accumulation):
 //                    S   = Q_i K_j^T    bf16  M=128 (q) N=64 (kv) K=d    A,B K-major
 //                    dP  = dO_i V_j^T   fp16  M=128 (q) N=64 (kv) K=d    A,B K-major
 //                    dV^T += dO_i^T P   fp16  M=d       N=64 (kv) K=128  A,B MN-major
 //                    dK^T += Q_i^T dS   bf16  M=d       N=64 (kv) K=128  A,B MN-major
-//                    dQ  = dS K_j       bf16  M=128 (q) N=d       K=64   A K-, B MN-major
 //                  Warps 0-7 turn S, dP into P (fp16: 11-bit significand, P in
 //                  [0, 1]) and dS (a hi + lo pair of bf16 tiles, about 16
-//                  significant bits, as dS feeds dQ and dK where a bf16 rounding
-//                  of it is amplified by large keys); warpgroup h (warps 4h ..
-//                  4h+3) handles kv columns 32h .. 32h+31, thread = query row.
-//                  The dK^T and dQ products run once per half of dS.
-//                  Warps 8-11 drain each dQ tile from TMEM through a shared-
-//                  memory staging tile into the fp32 dQ with TMA bulk
-//                  reduce-add (the output itself for fp32 gradients). Warp 12
-//                  is the TMA producer; warp 13 issues the MMAs and owns TMEM.
+//                  significant bits, since a bf16 rounding of dS is amplified by
+//                  large keys in dK and dQ); warpgroup h handles kv columns
+//                  32h .. 32h+31, thread = query row. The dK^T product runs once
+//                  per half of dS. Warp 8: TMA producer; warp 9: MMA issuer.
+// bwd_dq_kernel    one CTA per (q-block i, head), looping over the kv-blocks j
+//                  that i keeps (CSR row of i); recomputes S and dP, forms dS as
+//                  above and accumulates dQ_i = sum_j dS_ij K_j in TMEM
+//                    dQ  += dS K_j      bf16  M=128 (q) N=d       K=64   A K-, B MN-major
+//                  then writes it once: no atomics and no fp32 scratch for dQ.
 //                  For d = 64 the dV^T / dK^T MMAs still run at M = 128 (the
 //                  upper 64 lanes repeat the lower ones and are ignored).
-// dq_convert_kernel  fp32 dQ -> bf16 dQ (bf16 gradients only).
 //
-// TMEM columns: S[2] 0..127, dP[2] 128..255, dV^T 256..319, dK^T 320..383,
-// dQ 384..384+d.
+// TMEM columns (both kernels): S[2] 0..127, dP[2] 128..255; dV^T 256..319 and
+// dK^T 320..383 (dkdv), dQ 256..256+d (dq).
 #include <algorithm>
 
 #include "common.cuh"
@@ -41,7 +40,7 @@ namespace spa2 {
 
 namespace {
 
-constexpr int BWD_THREADS = 448;
+constexpr int BWD_THREADS = 320;  // P/dS x 8 warps, TMA, MMA
 
 template <int D>
 struct BwdSmem {
@@ -52,11 +51,9 @@ struct BwdSmem {
   alignas(1024) uint8_t dO[2][CH][128 * 128];    // dO_i fp16
   alignas(1024) uint8_t p[128 * 128];            // P  [128 q][64 kv] fp16
   alignas(1024) uint8_t ds[2][128 * 128];        // dS [128 q][64 kv]: hi, lo bf16 tiles
-  alignas(1024) uint8_t dq_stage[128 * 128];     // one 32-column fp32 slice of a dQ tile
   uint64_t kv_full;
   uint64_t qd_full[2], qd_empty[2], sdp_full[2];
-  uint64_t pds_full, pds_empty, dq_full, dq_empty, acc_done, drain;
-  uint64_t stage_full, stage_free;
+  uint64_t pds_full, pds_empty, acc_done, drain;
   uint32_t tmem_base;
   int abort_flag;
   int never;
@@ -65,15 +62,6 @@ struct BwdSmem {
 SPA2_DEV bool wait_warp(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
   const bool ok = wait_bar(bar, parity, w);
   return __all_sync(0xffffffff, ok);
-}
-
-// TMA bulk reduce-add of a shared-memory tile into global memory (fp32 add)
-SPA2_DEV void tma_reduce_add_3d(const CUtensorMap* map, const void* src, int c0, int c1, int c2) {
-  asm volatile(
-      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
-          reinterpret_cast<uint64_t>(map)),
-      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
-      : "memory");
 }
 
 // packed fp32 pairs (sm_100 f32x2 arithmetic): low half = first element
@@ -114,12 +102,11 @@ SPA2_DEV void split_bf16(float a, float b, uint32_t& hi, uint32_t& lo) {
 }  // namespace
 
 template <int D>
-__global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const __grid_constant__ CUtensorMap tm_q,
-                                                             const __grid_constant__ CUtensorMap tm_k,
-                                                             const __grid_constant__ CUtensorMap tm_v16,
-                                                             const __grid_constant__ CUtensorMap tm_do16,
-                                                             const __grid_constant__ CUtensorMap tm_dq,
-                                                             const float* __restrict__ lse,
+__global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                                                  const __grid_constant__ CUtensorMap tm_k,
+                                                                  const __grid_constant__ CUtensorMap tm_v16,
+                                                                  const __grid_constant__ CUtensorMap tm_do16,
+                                                                  const float* __restrict__ lse,
                                                              const float* __restrict__ dvec,
                                                              const int* __restrict__ col_cnt,
                                                              const int* __restrict__ col_idx, void* __restrict__ dk,
@@ -131,12 +118,11 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const __grid_consta
   constexpr uint32_t IDESC_DP = idesc_bf16_f32(128, 64, false, false, /*f16=*/true);
   constexpr uint32_t IDESC_DV = idesc_bf16_f32(128, 64, true, true, /*f16=*/true);
   constexpr uint32_t IDESC_T = idesc_bf16_f32(128, 64, true, true);
-  constexpr uint32_t IDESC_Q = idesc_bf16_f32(128, D, false, true);
   constexpr uint32_t QT_BYTES = 128 * D * 2;
   constexpr uint32_t KV_BYTES = 64 * D * 2;
   // MN-major A operand (dO^T, Q^T): stride between the two 64-row halves of M = d
   constexpr uint32_t LBO_DT = (D == 128) ? 128 * 128 : 0;
-  constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 320, T_DQ = 384;
+  constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 320;
   constexpr float LOG2E = 1.4426950408889634f;
 
   extern __shared__ uint8_t smem_raw[];
@@ -149,7 +135,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const __grid_consta
   const long long colid = (long long)bh * Tn + j;
   const int kv_valid = min(64, N - j * 64);
 
-  if (warp == 13) {
+  if (warp == 9) {
     tmem_alloc(&sm.tmem_base, 512);
     tmem_relinquish();
   }
@@ -162,12 +148,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const __grid_consta
     }
     mbar_init(&sm.pds_full, 256);
     mbar_init(&sm.pds_empty, 1);
-    mbar_init(&sm.dq_full, 1);
-    mbar_init(&sm.dq_empty, 128);
     mbar_init(&sm.acc_done, 1);
     mbar_init(&sm.drain, 1);
-    mbar_init(&sm.stage_full, 128);
-    mbar_init(&sm.stage_free, 1);
     sm.abort_flag = 0;
     sm.never = 0;
     fence_mbar_init();
@@ -186,7 +168,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const __grid_consta
   }
   const int* q_list = col_idx + colid * Tm;
 
-  if (warp == 12) {
+  if (warp == 8) {
     // ---------------- TMA producer ----------------
     if (lane == 0 && n > 0) {
       tma_prefetch_desc(&tm_q);
@@ -218,7 +200,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const __grid_consta
       for (int t = max(0, issued - 2); t < issued; ++t) wait_bar(&sm.qd_full[t & 1], (t >> 1) & 1, drain_wc);
       wait_bar(&sm.kv_full, 0, drain_wc);
     }
-  } else if (warp == 13) {
+  } else if (warp == 9) {
     // ---------------- MMA issuer ----------------
     if (lane == 0 && n > 0) {
       const uint32_t p_addr = smem_u32(sm.p), ds_addr = smem_u32(sm.ds[0]);
@@ -261,18 +243,6 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const __grid_consta
                        sdesc_sw128(ds_addr + part * (128 * 128) + kk * 2048, 0, 1024), IDESC_T,
                        (u > 0 || part > 0 || kk > 0) ? 1u : 0u);
             }
-            // dQ tile = (dS_hi + dS_lo) K_j, K = 64 kv rows; TMEM dQ must have been drained
-            if (u >= 1 && !wait_bar(&sm.dq_empty, (u - 1) & 1, wc)) break;
-            tc_fence_after();
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                mma_ss(tmem + T_DQ, sdesc_sw128(ds_addr + part * (128 * 128) + kk * 32, 16, 1024),
-                       sdesc_sw128(smem_u32(sm.k[0]) + kk * 2048, 64 * 128, 1024), IDESC_Q,
-                       (part > 0 || kk > 0) ? 1u : 0u);
-            }
-            mma_commit(&sm.dq_full);
             mma_commit(&sm.qd_empty[su]);
             mma_commit(&sm.pds_empty);
           }
@@ -282,54 +252,6 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const __grid_consta
       mma_commit(&sm.drain);
       wait_bar(&sm.drain, 0, drain_wc);
     }
-  } else if (warp >= 8) {
-    // ---------------- dQ drain, warps 8-11: TMEM -> smem slice -> TMA reduce-add ----------------
-    const int r = threadIdx.x - 256;
-    const bool issuer = r == 0;
-    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    int slices = 0;  // 32-column slices staged so far
-    bool ok = true;
-    for (int t = 0; t < n && ok; ++t) {
-      if (!wait_warp(&sm.dq_full, t & 1, wc)) break;
-      tc_fence_after();
-      const int i = q_list[t];
-#pragma unroll 1
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t vq[32];
-        tmem_ld32(tl + T_DQ + cc * 32, vq);
-        tmem_wait_ld();
-        if (cc == D / 32 - 1) {
-          tc_fence_before();
-          mbar_arrive(&sm.dq_empty);  // the TMEM dQ tile has been read
-        }
-        // the staging slice is free once the previous reduce has read it
-        if (slices > 0 && !wait_warp(&sm.stage_free, (slices - 1) & 1, wc)) {
-          ok = false;
-          break;
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          *reinterpret_cast<float4*>(sm.dq_stage + sw128_offset(r, u)) =
-              make_float4(__uint_as_float(vq[4 * u]) * scale, __uint_as_float(vq[4 * u + 1]) * scale,
-                          __uint_as_float(vq[4 * u + 2]) * scale, __uint_as_float(vq[4 * u + 3]) * scale);
-        fence_proxy_async_smem();
-        mbar_arrive(&sm.stage_full);
-        if (issuer) {
-          if (!wait_bar(&sm.stage_full, slices & 1, wc)) {
-            ok = false;
-          } else {
-            tma_reduce_add_3d(&tm_dq, sm.dq_stage, cc * 32, i * 128, bh);
-            tma_store_commit();
-            asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-            mbar_arrive(&sm.stage_free);
-          }
-        }
-        ++slices;
-        ok = __all_sync(0xffffffff, ok);
-        if (!ok) break;
-      }
-    }
-    if (issuer) tma_store_wait_all();  // every reduce has landed before the CTA ends
   } else {
     // ---------------- P / dS warps 0-7 ----------------
     const int h = warp >> 2;           // kv columns 32h .. 32h+31
@@ -453,21 +375,296 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_kernel(const __grid_consta
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 13) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
 }
 
-// D = rowsum(dO * (O + O_lo)) in fp32; zero the fp32 dQ row; fp16 copies of the
-// dO and V rows (|x| > 65504 clamped and reported). 16 threads per row.
+namespace {
+
+constexpr int DQ_THREADS = 320;  // P/dS x 8 warps, TMA, MMA
+constexpr int DQ_KS = 3;         // K / V ring slots
+
+template <int D>
+struct DqSmem {
+  static constexpr int CH = D / 64;
+  alignas(1024) uint8_t q[CH][128 * 128];          // Q_i bf16
+  alignas(1024) uint8_t dO[CH][128 * 128];         // dO_i fp16
+  alignas(1024) uint8_t k[DQ_KS][CH][64 * 128];    // K_j bf16
+  alignas(1024) uint8_t v[DQ_KS][CH][64 * 128];    // V_j fp16
+  alignas(1024) uint8_t ds[2][2][128 * 128];       // [buffer][hi, lo] dS [128 q][64 kv] bf16
+  uint64_t qd_full;
+  uint64_t kv_full[DQ_KS], kv_empty[DQ_KS];
+  uint64_t sdp_full[2], ds_full[2], ds_empty[2];
+  uint64_t acc_done, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int never;
+};
+
+}  // namespace
+
+template <int D>
+__global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                                               const __grid_constant__ CUtensorMap tm_k,
+                                                               const __grid_constant__ CUtensorMap tm_v16,
+                                                               const __grid_constant__ CUtensorMap tm_do16,
+                                                               const float* __restrict__ lse,
+                                                               const float* __restrict__ dvec,
+                                                               const int* __restrict__ row_cnt,
+                                                               const int* __restrict__ row_idx, void* __restrict__ dq,
+                                                               int grad_f32, int N, int Tm, int Tn, float scale,
+                                                               float scale_log2, int* status,
+                                                               unsigned long long wait_limit_ns) {
+  constexpr int CH = D / 64;
+  constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, false, false);
+  constexpr uint32_t IDESC_DP = idesc_bf16_f32(128, 64, false, false, /*f16=*/true);
+  constexpr uint32_t IDESC_Q = idesc_bf16_f32(128, D, false, true);
+  constexpr uint32_t QT_BYTES = 128 * D * 2;
+  constexpr uint32_t KV_BYTES = 64 * D * 2;
+  constexpr uint32_t T_S = 0, T_DP = 128, T_DQ = 256;
+  constexpr float LOG2E = 1.4426950408889634f;
+
+  extern __shared__ uint8_t smem_raw[];
+  DqSmem<D>& sm = *reinterpret_cast<DqSmem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+  const int warp = threadIdx.x >> 5;
+  const uint32_t lane = lane_id();
+  const int i = blockIdx.x;
+  const int bh = blockIdx.y;
+  const long long rowid = (long long)bh * Tm + i;
+
+  if (warp == 9) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 256) {
+    mbar_init(&sm.qd_full, 1);
+    for (int x = 0; x < DQ_KS; ++x) {
+      mbar_init(&sm.kv_full[x], 1);
+      mbar_init(&sm.kv_empty[x], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.sdp_full[b], 1);
+      mbar_init(&sm.ds_full[b], 256);
+      mbar_init(&sm.ds_empty[b], 1);
+    }
+    mbar_init(&sm.acc_done, 1);
+    mbar_init(&sm.drain, 1);
+    sm.abort_flag = 0;
+    sm.never = 0;
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const WaitCtx wc{&sm.abort_flag, status, wait_limit_ns};
+  const WaitCtx drain_wc{&sm.never, nullptr, wait_limit_ns};
+
+  int n = row_cnt[rowid];
+  if (n < 1 || n > Tn) {
+    if (threadIdx.x == 0) report(status, SPA2_ERR_DEVICE_BOUNDS);
+    n = 0;
+  }
+  const int* kv_list = row_idx + rowid * Tn;
+
+  if (warp == 8) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0 && n > 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v16);
+      tma_prefetch_desc(&tm_do16);
+      mbar_expect_tx(&sm.qd_full, 2 * QT_BYTES);
+      for (int c = 0; c < CH; ++c) {
+        tma_load_3d(sm.q[c], &tm_q, &sm.qd_full, c * 64, i * 128, bh);
+        tma_load_3d(sm.dO[c], &tm_do16, &sm.qd_full, c * 64, i * 128, bh);
+      }
+      int issued = 0;
+      for (int t = 0; t < n; ++t) {
+        const int slot = t % DQ_KS;
+        if (t >= DQ_KS && !wait_bar(&sm.kv_empty[slot], ((t / DQ_KS) - 1) & 1, wc)) break;
+        const int j = kv_list[t];
+        if (j < 0 || j >= Tn) {
+          report(status, SPA2_ERR_DEVICE_BOUNDS);
+          sm.abort_flag = 1;
+          break;
+        }
+        mbar_expect_tx(&sm.kv_full[slot], 2 * KV_BYTES);
+        for (int c = 0; c < CH; ++c) {
+          tma_load_3d(sm.k[slot][c], &tm_k, &sm.kv_full[slot], c * 64, j * 64, bh);
+          tma_load_3d(sm.v[slot][c], &tm_v16, &sm.kv_full[slot], c * 64, j * 64, bh);
+        }
+        issued = t + 1;
+      }
+      for (int t = max(0, issued - DQ_KS); t < issued; ++t)
+        wait_bar(&sm.kv_full[t % DQ_KS], (t / DQ_KS) & 1, drain_wc);
+      wait_bar(&sm.qd_full, 0, drain_wc);
+    }
+  } else if (warp == 9) {
+    // ---------------- MMA issuer: S(t), dP(t), then dQ += dS(t-1) K(t-1) ----------------
+    if (lane == 0 && n > 0) {
+      const uint32_t qa = smem_u32(sm.q[0]), da = smem_u32(sm.dO[0]);
+      if (wait_bar(&sm.qd_full, 0, wc)) {
+        for (int t = 0; t <= n; ++t) {
+          if (t < n) {
+            const int b = t & 1, slot = t % DQ_KS;
+            if (!wait_bar(&sm.kv_full[slot], (t / DQ_KS) & 1, wc)) break;
+            tc_fence_after();
+            const uint32_t kb = smem_u32(sm.k[slot][0]), vb = smem_u32(sm.v[slot][0]);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * (64 * 128) + (kk & 3) * 32;
+              const uint32_t offq = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+              mma_ss(tmem + T_S + b * 64, sdesc_sw128(qa + offq, 16, 1024), sdesc_sw128(kb + off, 16, 1024), IDESC_S,
+                     kk > 0 ? 1u : 0u);
+            }
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * (64 * 128) + (kk & 3) * 32;
+              const uint32_t offq = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+              mma_ss(tmem + T_DP + b * 64, sdesc_sw128(da + offq, 16, 1024), sdesc_sw128(vb + off, 16, 1024),
+                     IDESC_DP, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(&sm.sdp_full[b]);
+          }
+          if (t >= 1) {
+            const int u = t - 1, b = u & 1, slot = u % DQ_KS;
+            if (!wait_bar(&sm.ds_full[b], (u >> 1) & 1, wc)) break;
+            tc_fence_after();
+            const uint32_t dsa = smem_u32(sm.ds[b][0]), kb = smem_u32(sm.k[slot][0]);
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                mma_ss(tmem + T_DQ, sdesc_sw128(dsa + part * (128 * 128) + kk * 32, 16, 1024),
+                       sdesc_sw128(kb + kk * 2048, 64 * 128, 1024), IDESC_Q, (u > 0 || part > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(&sm.ds_empty[b]);
+            mma_commit(&sm.kv_empty[slot]);
+          }
+        }
+        mma_commit(&sm.acc_done);
+      }
+      mma_commit(&sm.drain);
+      wait_bar(&sm.drain, 0, drain_wc);
+    }
+  } else {
+    // ---------------- dS warps 0-7: warpgroup h handles kv columns 32h .. 32h+31 ----------------
+    const int h = warp >> 2;
+    const int r = threadIdx.x & 127;  // query row == TMEM lane
+    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const long long row = (long long)i * 128 + r;
+    const bool rvalid = row < N;
+    const float nlse2 = rvalid ? -lse[(long long)bh * N + row] * LOG2E : -INFINITY;
+    const float Dr = rvalid ? dvec[(long long)bh * N + row] : 0.f;
+    const uint64_t scale2 = f2_pack(scale_log2, scale_log2), nlse2x2 = f2_pack(nlse2, nlse2),
+                   d2 = f2_pack(Dr, Dr);
+    // only kv-block Tn-1 (last in the ascending list) is ragged
+    const int last_valid = (n > 0 && kv_list[n - 1] == Tn - 1) ? N - (Tn - 1) * 64 : 64;
+    bool ok = n > 0;
+    for (int t = 0; t < n && ok; ++t) {
+      const int b = t & 1;
+      if (!wait_warp(&sm.sdp_full[b], (t >> 1) & 1, wc)) {
+        ok = false;
+        break;
+      }
+      // this dS buffer was read by the dQ product of tile t-2
+      if (t >= 2 && !wait_warp(&sm.ds_empty[b], ((t - 2) >> 1) & 1, wc)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int kv_valid = t == n - 1 ? last_valid : 64;
+#pragma unroll
+      for (int sub = 0; sub < 2; ++sub) {
+        const int c0 = h * 32 + sub * 16;
+        uint32_t sa[16], pa[16];
+        tmem_ld16(tl + T_S + b * 64 + c0, sa);
+        tmem_ld16(tl + T_DP + b * 64 + c0, pa);
+        tmem_wait_ld();
+        uint32_t dh[8], dl[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sa[2 * e]), __uint_as_float(sa[2 * e + 1])), scale2,
+                                     nlse2x2);
+          float x0, x1;
+          f2_unpack(x2, x0, x1);
+          float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+          if (kv_valid < 64) {
+            if (c0 + 2 * e >= kv_valid) p0 = 0.f;
+            if (c0 + 2 * e + 1 >= kv_valid) p1 = 0.f;
+          }
+          const uint64_t ds2 = f2_mul(f2_pack(p0, p1),
+                                      f2_sub(f2_pack(__uint_as_float(pa[2 * e]), __uint_as_float(pa[2 * e + 1])), d2));
+          float s0, s1;
+          f2_unpack(ds2, s0, s1);
+          split_bf16(s0, s1, dh[e], dl[e]);
+        }
+        const uint32_t u0 = c0 >> 3;
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          const uint32_t off = sw128_offset(r, u0 + w);
+          *reinterpret_cast<uint4*>(sm.ds[b][0] + off) =
+              make_uint4(dh[4 * w], dh[4 * w + 1], dh[4 * w + 2], dh[4 * w + 3]);
+          *reinterpret_cast<uint4*>(sm.ds[b][1] + off) =
+              make_uint4(dl[4 * w], dl[4 * w + 1], dl[4 * w + 2], dl[4 * w + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&sm.ds_full[b]);
+    }
+    // epilogue: dQ_i = scale * acc; warpgroup h writes feature columns h*D/2 .. +D/2
+    if (ok) ok = wait_warp(&sm.acc_done, 0, wc);
+    if (ok) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int cc = 0; cc < D / 64; ++cc) {
+        const int c0 = h * (D / 2) + cc * 32;
+        uint32_t a[32];
+        tmem_ld32(tl + T_DQ + c0, a);
+        tmem_wait_ld();
+        if (rvalid) {
+          const long long base = ((long long)bh * N + row) * D + c0;
+          if (grad_f32) {
+            float4* o = reinterpret_cast<float4*>(static_cast<float*>(dq) + base);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              o[e] = make_float4(__uint_as_float(a[4 * e]) * scale, __uint_as_float(a[4 * e + 1]) * scale,
+                                 __uint_as_float(a[4 * e + 2]) * scale, __uint_as_float(a[4 * e + 3]) * scale);
+          } else {
+            uint4* o = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dq) + base);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              o[e] = make_uint4(pack_bf16(__uint_as_float(a[8 * e]) * scale, __uint_as_float(a[8 * e + 1]) * scale),
+                                pack_bf16(__uint_as_float(a[8 * e + 2]) * scale, __uint_as_float(a[8 * e + 3]) * scale),
+                                pack_bf16(__uint_as_float(a[8 * e + 4]) * scale, __uint_as_float(a[8 * e + 5]) * scale),
+                                pack_bf16(__uint_as_float(a[8 * e + 6]) * scale, __uint_as_float(a[8 * e + 7]) * scale));
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// D = rowsum(dO * (O + O_lo)) in fp32; fp16 copies of the dO and V rows
+// (|x| > 65504 clamped and reported). 16 threads per row.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
                                                       const __nv_bfloat16* __restrict__ o_lo,
                                                       const __nv_bfloat16* __restrict__ dout,
                                                       const __nv_bfloat16* __restrict__ v,
-                                                      float* __restrict__ dvec, float* __restrict__ dq32,
-                                                      uint32_t* __restrict__ do16, uint32_t* __restrict__ v16,
+                                                      float* __restrict__ dvec, uint32_t* __restrict__ do16, uint32_t* __restrict__ v16,
                                                       long long rows, int* status) {
   constexpr int TPR = 16;
   constexpr int EPT = D / TPR;  // 8 (d=128) or 4 (d=64) elements per thread
@@ -500,9 +697,6 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __res
       do16[(off + e) / 2] = pack_f16(b.x, b.y);
       v16[(off + e) / 2] = pack_f16(w.x, w.y);
     }
-    float4* z = reinterpret_cast<float4*>(dq32 + off);
-#pragma unroll
-    for (int e = 0; e < EPT / 4; ++e) z[e] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
 #pragma unroll
   for (int s = TPR / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffff, acc, s);
@@ -510,57 +704,41 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __res
   if (bad) report(status, SPA2_ERR_RANGE);
 }
 
-__global__ void __launch_bounds__(256) dq_convert_kernel(const float4* __restrict__ src, uint2* __restrict__ dst,
-                                                         long long n4) {
-  for (long long e = (long long)blockIdx.x * 256 + threadIdx.x; e < n4; e += (long long)gridDim.x * 256) {
-    const float4 v = src[e];
-    dst[e] = make_uint2(pack_bf16(v.x, v.y), pack_bf16(v.z, v.w));
-  }
-}
-
 template <int D>
-static cudaError_t launch_bwd_main(const BwdArgs& a, float* dq32, cudaStream_t s) {
-  (void)dq32;
-  const size_t smem = sizeof(BwdSmem<D>) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+static cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
+  const long long rows = (long long)a.BH * a.N;
+  // 1. D and the fp16 copies of dO and V
+  bwd_pre_kernel<D><<<(unsigned)((rows + 15) / 16), 256, 0, s>>>(
+      (const __nv_bfloat16*)a.o, (const __nv_bfloat16*)a.o_lo, (const __nv_bfloat16*)a.dout,
+      (const __nv_bfloat16*)a.v, a.dvec, (uint32_t*)a.do16, (uint32_t*)a.v16, rows, a.status);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  dim3 grid(a.Tn, a.BH);
-  bwd_kernel<D><<<grid, BWD_THREADS, smem, s>>>(*a.tm_q, *a.tm_k, *a.tm_v, *a.tm_do, *a.tm_dq, a.lse, a.dvec,
-                                                a.col_cnt, a.col_idx, a.dk, a.dv, a.grad_f32, a.N, a.Tm, a.Tn,
-                                                a.scale, a.scale_log2, a.status, a.wait_limit_ns);
-  return cudaGetLastError();
+  // 2. dK, dV (kv-major)
+  {
+    const size_t smem = sizeof(BwdSmem<D>) + 1024;
+    e = cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    bwd_dkdv_kernel<D><<<dim3(a.Tn, a.BH), BWD_THREADS, smem, s>>>(
+        *a.tm_q, *a.tm_k, *a.tm_v, *a.tm_do, a.lse, a.dvec, a.col_cnt, a.col_idx, a.dk, a.dv, a.grad_f32, a.N, a.Tm,
+        a.Tn, a.scale, a.scale_log2, a.status, a.wait_limit_ns);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  // 3. dQ (q-major)
+  {
+    const size_t smem = sizeof(DqSmem<D>) + 1024;
+    e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    bwd_dq_kernel<D><<<dim3(a.Tm, a.BH), DQ_THREADS, smem, s>>>(
+        *a.tm_q, *a.tm_k, *a.tm_v, *a.tm_do, a.lse, a.dvec, a.row_cnt, a.row_idx, a.dq, a.grad_f32, a.N, a.Tm,
+        a.Tn, a.scale, a.scale_log2, a.status, a.wait_limit_ns);
+    e = cudaGetLastError();
+  }
+  return e;
 }
 
 cudaError_t launch_bwd(const BwdArgs& a, int d, cudaStream_t s) {
-  const long long rows = (long long)a.BH * a.N;
-  float* dq32 = a.grad_f32 ? static_cast<float*>(a.dq) : a.dq_acc;
-  // 1. D, dQ reset, fp16 copies of dO and V
-  {
-    dim3 grid((unsigned)((rows + 15) / 16));
-    if (d == 128)
-      bwd_pre_kernel<128><<<grid, 256, 0, s>>>((const __nv_bfloat16*)a.o, (const __nv_bfloat16*)a.o_lo,
-                                               (const __nv_bfloat16*)a.dout, (const __nv_bfloat16*)a.v, a.dvec,
-                                               dq32, (uint32_t*)a.do16, (uint32_t*)a.v16, rows, a.status);
-    else
-      bwd_pre_kernel<64><<<grid, 256, 0, s>>>((const __nv_bfloat16*)a.o, (const __nv_bfloat16*)a.o_lo,
-                                              (const __nv_bfloat16*)a.dout, (const __nv_bfloat16*)a.v, a.dvec,
-                                              dq32, (uint32_t*)a.do16, (uint32_t*)a.v16, rows, a.status);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
-  // 2. main kernel
-  {
-    cudaError_t e = d == 128 ? launch_bwd_main<128>(a, dq32, s) : launch_bwd_main<64>(a, dq32, s);
-    if (e != cudaSuccess) return e;
-  }
-  // 3. dQ fp32 -> bf16
-  if (!a.grad_f32) {
-    const long long n4 = rows * d / 4;
-    const unsigned blocks = (unsigned)std::min<long long>((n4 + 255) / 256, 148LL * 16);
-    dq_convert_kernel<<<blocks, 256, 0, s>>>((const float4*)a.dq_acc, (uint2*)a.dq, n4);
-    return cudaGetLastError();
-  }
-  return cudaSuccess;
+  return d == 128 ? launch_bwd_d<128>(a, s) : launch_bwd_d<64>(a, s);
 }
 
 }  // namespace spa2

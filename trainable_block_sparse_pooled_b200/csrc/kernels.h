@@ -49,22 +49,22 @@ struct BwdArgs {
   const CUtensorMap* tm_k;    // K bf16, box {64, 64, 1}
   const CUtensorMap* tm_v;    // fp16 copy of V, box {64, 64, 1}
   const CUtensorMap* tm_do;   // fp16 copy of dO, box {64, 128, 1}
-  const CUtensorMap* tm_dq;   // fp32 dQ accumulator, box {32, 128, 1}
   const void* o;
   const void* o_lo;   // may be null
   const void* dout;
   const void* v;
   const float* lse;
+  const int* row_cnt;
+  const int* row_idx;
   const int* col_cnt;
   const int* col_idx;
   float* dvec;     // [BH, N]
-  float* dq_acc;   // [BH, N, d]
   void* do16;      // [BH, N, d] fp16
   void* v16;       // [BH, N, d] fp16
   void* dq;
   void* dk;
   void* dv;
-  int grad_f32;       // 1: dq/dk/dv are fp32 (dQ accumulates in place), 0: bf16
+  int grad_f32;       // 1: dq/dk/dv are fp32, 0: bf16
   int BH, N, Tm, Tn;
   float scale;        // softmax_scale
   float scale_log2;   // softmax_scale * log2(e)
