@@ -46,6 +46,29 @@ WORKLOADS = {
 }
 
 
+def profiled_traffic(workload):
+    """DRAM bytes (read + write) of one backward call on this workload, from the
+    ncu summary under profiles/, or None when the summary is missing, covers
+    another workload, or was taken on a different backward source."""
+    import hashlib
+    here = os.path.dirname(os.path.abspath(__file__))
+    path = os.path.join(here, "profiles", "bwd_traffic.txt")
+    src = os.path.join(here, "trainable_block_sparse_pooled_b200", "csrc", "attn_bwd.cu")
+    try:
+        fields = dict(line.split(":", 1) for line in open(path, encoding="utf-8")
+                      if ":" in line and not line.startswith("#"))
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    fields = {k.strip(): v.strip() for k, v in fields.items()}
+    if fields.get("source_sha256") != sha or fields.get("workload") != workload:
+        return None
+    try:
+        return int(fields["bytes_per_call"])
+    except (KeyError, ValueError):
+        return None
+
+
 def peaks():
     try:
         with open(PEAKS_FILE) as f:
@@ -301,7 +324,7 @@ def run_gpu(args, wl, name):
     dq = torch.empty(q.shape, dtype=gt, device=dev)
     dk = torch.empty(q.shape, dtype=gt, device=dev)
     dv = torch.empty(q.shape, dtype=gt, device=dev)
-    launches_per_step = 3 + 2 + 2   # pool, pbar+select, csc | V->fp16, fwd | D/zero, bwd
+    launches_per_step = 3 + 2 + 3   # pool, select, csc | V->fp16, fwd | D + fp16 copies, dK/dV, dQ
 
     def step(ev=None):
         if ev is not None:
@@ -416,9 +439,9 @@ def run_gpu(args, wl, name):
                              "seeded N(0,1) with 2 sink keys, dO ~ N(0,1)",
                    "grad_dtype": "fp32", "l2": "inputs larger than L2 (Q, K, V, dO are 4 x %.0f MB)" %
                    (B * H * N * d * 2 / 1e6), "parallelism": f"independent layer per GPU x{ws}"},
-        "roofline": {"bound": "tensor", "kernel": "bwd (D pre-pass + bwd_kernel)", "achieved": bwd_tf,
-                     "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                     "frac": bwd_tf / pk["bf16_tflops_sustained"], "traffic": None,
+        "roofline": {"bound": "tensor", "kernel": "backward call: D pre-pass + bwd_dkdv_kernel + bwd_dq_kernel",
+                     "achieved": bwd_tf, "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                     "frac": bwd_tf / pk["bf16_tflops_sustained"], "traffic": profiled_traffic(name),
                      "peak_kind": f"{pk_kind} bf16 sustained (kernel timed inside a long step)"},
         "cpu_baseline": cpu,
         "e2e": e2e,
@@ -449,13 +472,19 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the k = 100%% comparison pass")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override the workload's head count (a smaller case of the same layer, for profiling)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    wl = WORKLOADS[args.workload]
+    wl = dict(WORKLOADS[args.workload])
+    name = args.workload
+    if args.heads > 0:
+        wl["H"] = args.heads
+        name = f"{args.workload} ({args.heads} heads)"
     if args.impl == "reference":
-        return run_reference(args, wl, args.workload)
-    return run_gpu(args, wl, args.workload)
+        return run_reference(args, wl, name)
+    return run_gpu(args, wl, name)
 
 
 if __name__ == "__main__":
