@@ -204,50 +204,65 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
     // ---------------- MMA issuer ----------------
     if (lane == 0 && n > 0) {
       const uint32_t p_addr = smem_u32(sm.p), ds_addr = smem_u32(sm.ds[0]);
-      if (wait_bar(&sm.kv_full, 0, wc)) {
-        for (int t = 0; t <= n; ++t) {
-          if (t < n) {
-            const int s = t & 1;
-            if (!wait_bar(&sm.qd_full[s], (t >> 1) & 1, wc)) break;
-            tc_fence_after();
+      // S(t), dP(t) into TMEM buffer t mod 2 (Q / dO stage t mod 2)
+      auto issue_sdp = [&](int t) {
+        const int s = t & 1;
+        tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * (64 * 128) + (kk & 3) * 32;
-              const uint32_t offq = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-              mma_ss(tmem + T_S + s * 64, sdesc_sw128(smem_u32(sm.q[s][0]) + offq, 16, 1024),
-                     sdesc_sw128(smem_u32(sm.k[0]) + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
-            }
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (64 * 128) + (kk & 3) * 32;
+          const uint32_t offq = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+          mma_ss(tmem + T_S + s * 64, sdesc_sw128(smem_u32(sm.q[s][0]) + offq, 16, 1024),
+                 sdesc_sw128(smem_u32(sm.k[0]) + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+        }
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * (64 * 128) + (kk & 3) * 32;
-              const uint32_t offq = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-              mma_ss(tmem + T_DP + s * 64, sdesc_sw128(smem_u32(sm.dO[s][0]) + offq, 16, 1024),
-                     sdesc_sw128(smem_u32(sm.v[0]) + off, 16, 1024), IDESC_DP, kk > 0 ? 1u : 0u);
-            }
-            mma_commit(&sm.sdp_full[s]);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (64 * 128) + (kk & 3) * 32;
+          const uint32_t offq = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+          mma_ss(tmem + T_DP + s * 64, sdesc_sw128(smem_u32(sm.dO[s][0]) + offq, 16, 1024),
+                 sdesc_sw128(smem_u32(sm.v[0]) + off, 16, 1024), IDESC_DP, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&sm.sdp_full[s]);
+      };
+      // S/dP(u+1) goes ahead of dV/dK(u) only when its Q / dO tile has already
+      // landed; a late tile never holds back the products the P / dS warps wait on
+      int T = 0;  // S/dP issued
+      bool ok = wait_bar(&sm.kv_full, 0, wc) && wait_bar(&sm.qd_full[0], 0, wc);
+      if (ok) {
+        issue_sdp(0);
+        T = 1;
+        for (int u = 0; u < n && ok; ++u) {
+          if (T == u + 1 && T < n && mbar_test_wait(&sm.qd_full[T & 1], (T >> 1) & 1)) issue_sdp(T++);
+          const int su = u & 1;
+          if (!wait_bar(&sm.pds_full, u & 1, wc)) {
+            ok = false;
+            break;
           }
-          if (t >= 1) {
-            const int u = t - 1, su = u & 1;
-            if (!wait_bar(&sm.pds_full, u & 1, wc)) break;
-            tc_fence_after();
-            // dV^T += dO^T P (fp16); dK^T += Q^T (dS_hi + dS_lo) (bf16); K = 128 query rows
+          tc_fence_after();
+          // dV^T += dO^T P (fp16); dK^T += Q^T (dS_hi + dS_lo) (bf16); K = 128 query rows
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tmem + T_DV, sdesc_sw128(smem_u32(sm.dO[su][0]) + kk * 2048, LBO_DT, 1024),
+                   sdesc_sw128(p_addr + kk * 2048, 0, 1024), IDESC_DV, (u > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int part = 0; part < 2; ++part) {
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-              mma_ss(tmem + T_DV, sdesc_sw128(smem_u32(sm.dO[su][0]) + kk * 2048, LBO_DT, 1024),
-                     sdesc_sw128(p_addr + kk * 2048, 0, 1024), IDESC_DV, (u > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-#pragma unroll
-              for (int kk = 0; kk < 8; ++kk)
-                mma_ss(tmem + T_DK, sdesc_sw128(smem_u32(sm.q[su][0]) + kk * 2048, LBO_DT, 1024),
-                       sdesc_sw128(ds_addr + part * (128 * 128) + kk * 2048, 0, 1024), IDESC_T,
-                       (u > 0 || part > 0 || kk > 0) ? 1u : 0u);
+              mma_ss(tmem + T_DK, sdesc_sw128(smem_u32(sm.q[su][0]) + kk * 2048, LBO_DT, 1024),
+                     sdesc_sw128(ds_addr + part * (128 * 128) + kk * 2048, 0, 1024), IDESC_T,
+                     (u > 0 || part > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&sm.qd_empty[su]);
+          mma_commit(&sm.pds_empty);
+          if (T == u + 1 && T < n) {
+            if (!wait_bar(&sm.qd_full[T & 1], (T >> 1) & 1, wc)) {
+              ok = false;
+              break;
             }
-            mma_commit(&sm.qd_empty[su]);
-            mma_commit(&sm.pds_empty);
+            issue_sdp(T++);
           }
         }
-        mma_commit(&sm.acc_done);
+        if (ok) mma_commit(&sm.acc_done);
       }
       mma_commit(&sm.drain);
       wait_bar(&sm.drain, 0, drain_wc);

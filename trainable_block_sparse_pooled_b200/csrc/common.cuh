@@ -81,6 +81,19 @@ SPA2_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// non-blocking probe: has the phase of the given parity completed?
+SPA2_DEV bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Per-CTA abort flag + time limit. A wait that runs past the limit records
 // SPA2_ERR_DEVICE_TIMEOUT, raises the CTA's abort flag and returns false; every
 // other wait in the CTA then gives up at once, so the CTA reaches its teardown
