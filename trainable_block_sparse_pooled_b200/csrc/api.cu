@@ -296,7 +296,7 @@ spa2_status spa2_sparse_attn_bwd(const void* q, const void* k, const void* v, co
       !make_map(&tdo, w.do16, s, 128, true))
     return SPA2_ERR_CUDA;
   SPA2_CUDA_TRY(cudaMemsetAsync(w.status, 0, 4, st));
-  BwdArgs a{&tq, &tk, &tv, &tdo, o, o_lo, dout, v, lse, mask->row_cnt, mask->row_idx, mask->col_cnt,
+  BwdArgs a{&tq, &tk, &tv, &tdo, q, o, o_lo, dout, v, lse, mask->row_cnt, mask->row_idx, mask->col_cnt,
             mask->col_idx, w.dvec, w.do16, w.v16, dq, dk, dv, f32 ? 1 : 0, (int)s.BH, s.N, s.Tm, s.Tn, scale,
             scale * 1.4426950408889634f, w.status, g_wait_limit_ns};
   SPA2_CUDA_TRY(launch_bwd(a, d, st));

@@ -398,20 +398,17 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
 
 namespace {
 
-constexpr int DQ_THREADS = 320;  // P/dS x 8 warps, TMA, MMA
-constexpr int DQ_KS = 3;         // K / V ring slots
+constexpr int DQ_THREADS = 320;  // dS x 8 warps, TMA, MMA
+constexpr int DQ_KS = 6;         // K / V ring slots
 
 template <int D>
 struct DqSmem {
   static constexpr int CH = D / 64;
-  alignas(1024) uint8_t q[CH][128 * 128];          // Q_i bf16
-  alignas(1024) uint8_t dO[CH][128 * 128];         // dO_i fp16
   alignas(1024) uint8_t k[DQ_KS][CH][64 * 128];    // K_j bf16
   alignas(1024) uint8_t v[DQ_KS][CH][64 * 128];    // V_j fp16
-  alignas(1024) uint8_t ds[2][2][128 * 128];       // [buffer][hi, lo] dS [128 q][64 kv] bf16
-  uint64_t qd_full;
+  uint64_t qd_ready;
   uint64_t kv_full[DQ_KS], kv_empty[DQ_KS];
-  uint64_t sdp_full[2], ds_full[2], ds_empty[2];
+  uint64_t sdp_full[2], ds_full[2];
   uint64_t acc_done, drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -420,11 +417,18 @@ struct DqSmem {
 
 }  // namespace
 
+// Shared memory only holds the streamed K_j / V_j: Q_i and dO_i sit in TMEM as
+// the A operands of S and dP, and dS goes back into TMEM (over the S columns it
+// was computed from) as the A operand of dQ, so every product reads one
+// operand from shared memory (an SS product of these shapes is bound by the
+// 128 bytes per cycle the tensor core can read from shared memory).
+// TMEM columns: S[b] 64b .. 64b+63 (dS hi/lo of kv columns 32h .. 32h+31 go to
+// 64b+32h .. +15 / +16 .. +31), dP[b] 128+64b, dQ 256 .. 256+d, Q 384, dO 448.
 template <int D>
-__global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
-                                                               const __grid_constant__ CUtensorMap tm_k,
+__global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k,
                                                                const __grid_constant__ CUtensorMap tm_v16,
-                                                               const __grid_constant__ CUtensorMap tm_do16,
+                                                               const __nv_bfloat16* __restrict__ qg,
+                                                               const __half* __restrict__ do16,
                                                                const float* __restrict__ lse,
                                                                const float* __restrict__ dvec,
                                                                const int* __restrict__ row_cnt,
@@ -436,9 +440,8 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_cons
   constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, false, false);
   constexpr uint32_t IDESC_DP = idesc_bf16_f32(128, 64, false, false, /*f16=*/true);
   constexpr uint32_t IDESC_Q = idesc_bf16_f32(128, D, false, true);
-  constexpr uint32_t QT_BYTES = 128 * D * 2;
   constexpr uint32_t KV_BYTES = 64 * D * 2;
-  constexpr uint32_t T_S = 0, T_DP = 128, T_DQ = 256;
+  constexpr uint32_t T_S = 0, T_DP = 128, T_DQ = 256, T_Q = 384, T_DO = 448;
   constexpr float LOG2E = 1.4426950408889634f;
 
   extern __shared__ uint8_t smem_raw[];
@@ -455,7 +458,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_cons
     tmem_relinquish();
   }
   if (threadIdx.x == 256) {
-    mbar_init(&sm.qd_full, 1);
+    mbar_init(&sm.qd_ready, 256);
     for (int x = 0; x < DQ_KS; ++x) {
       mbar_init(&sm.kv_full[x], 1);
       mbar_init(&sm.kv_empty[x], 1);
@@ -463,7 +466,6 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_cons
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.sdp_full[b], 1);
       mbar_init(&sm.ds_full[b], 256);
-      mbar_init(&sm.ds_empty[b], 1);
     }
     mbar_init(&sm.acc_done, 1);
     mbar_init(&sm.drain, 1);
@@ -486,17 +488,10 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_cons
   const int* kv_list = row_idx + rowid * Tn;
 
   if (warp == 8) {
-    // ---------------- TMA producer ----------------
+    // ---------------- TMA producer: the K / V ring ----------------
     if (lane == 0 && n > 0) {
-      tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v16);
-      tma_prefetch_desc(&tm_do16);
-      mbar_expect_tx(&sm.qd_full, 2 * QT_BYTES);
-      for (int c = 0; c < CH; ++c) {
-        tma_load_3d(sm.q[c], &tm_q, &sm.qd_full, c * 64, i * 128, bh);
-        tma_load_3d(sm.dO[c], &tm_do16, &sm.qd_full, c * 64, i * 128, bh);
-      }
       int issued = 0;
       for (int t = 0; t < n; ++t) {
         const int slot = t % DQ_KS;
@@ -516,13 +511,11 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_cons
       }
       for (int t = max(0, issued - DQ_KS); t < issued; ++t)
         wait_bar(&sm.kv_full[t % DQ_KS], (t / DQ_KS) & 1, drain_wc);
-      wait_bar(&sm.qd_full, 0, drain_wc);
     }
   } else if (warp == 9) {
-    // ---------------- MMA issuer: S(t), dP(t), then dQ += dS(t-1) K(t-1) ----------------
+    // ---------------- MMA issuer: S(t), dP(t), then dQ += dS(t-1) K(t-1), all TS ----------------
     if (lane == 0 && n > 0) {
-      const uint32_t qa = smem_u32(sm.q[0]), da = smem_u32(sm.dO[0]);
-      if (wait_bar(&sm.qd_full, 0, wc)) {
+      if (wait_bar(&sm.qd_ready, 0, wc)) {
         for (int t = 0; t <= n; ++t) {
           if (t < n) {
             const int b = t & 1, slot = t % DQ_KS;
@@ -532,16 +525,14 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_cons
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t off = (kk >> 2) * (64 * 128) + (kk & 3) * 32;
-              const uint32_t offq = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-              mma_ss(tmem + T_S + b * 64, sdesc_sw128(qa + offq, 16, 1024), sdesc_sw128(kb + off, 16, 1024), IDESC_S,
+              mma_ts(tmem + T_S + b * 64, tmem + T_Q + kk * 8, sdesc_sw128(kb + off, 16, 1024), IDESC_S,
                      kk > 0 ? 1u : 0u);
             }
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t off = (kk >> 2) * (64 * 128) + (kk & 3) * 32;
-              const uint32_t offq = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-              mma_ss(tmem + T_DP + b * 64, sdesc_sw128(da + offq, 16, 1024), sdesc_sw128(vb + off, 16, 1024),
-                     IDESC_DP, kk > 0 ? 1u : 0u);
+              mma_ts(tmem + T_DP + b * 64, tmem + T_DO + kk * 8, sdesc_sw128(vb + off, 16, 1024), IDESC_DP,
+                     kk > 0 ? 1u : 0u);
             }
             mma_commit(&sm.sdp_full[b]);
           }
@@ -549,15 +540,14 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_cons
             const int u = t - 1, b = u & 1, slot = u % DQ_KS;
             if (!wait_bar(&sm.ds_full[b], (u >> 1) & 1, wc)) break;
             tc_fence_after();
-            const uint32_t dsa = smem_u32(sm.ds[b][0]), kb = smem_u32(sm.k[slot][0]);
+            const uint32_t kb = smem_u32(sm.k[slot][0]);
 #pragma unroll
             for (int part = 0; part < 2; ++part) {
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
-                mma_ss(tmem + T_DQ, sdesc_sw128(dsa + part * (128 * 128) + kk * 32, 16, 1024),
+                mma_ts(tmem + T_DQ, tmem + T_S + b * 64 + (kk >> 1) * 32 + part * 16 + (kk & 1) * 8,
                        sdesc_sw128(kb + kk * 2048, 64 * 128, 1024), IDESC_Q, (u > 0 || part > 0 || kk > 0) ? 1u : 0u);
             }
-            mma_commit(&sm.ds_empty[b]);
             mma_commit(&sm.kv_empty[slot]);
           }
         }
@@ -573,6 +563,27 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_cons
     const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const long long row = (long long)i * 128 + r;
     const bool rvalid = row < N;
+    // Q_i (warpgroup 0) and dO_i (warpgroup 1) into TMEM, one row per thread
+    {
+      const uint4* src = h == 0 ? reinterpret_cast<const uint4*>(qg + ((long long)bh * N + row) * D)
+                                : reinterpret_cast<const uint4*>(do16 + ((long long)bh * N + row) * D);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t w[32];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const uint4 x = rvalid ? src[c * 8 + e] : make_uint4(0, 0, 0, 0);
+          w[4 * e] = x.x;
+          w[4 * e + 1] = x.y;
+          w[4 * e + 2] = x.z;
+          w[4 * e + 3] = x.w;
+        }
+        tmem_st32(tl + (h == 0 ? T_Q : T_DO) + c * 32, w);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&sm.qd_ready);
+    }
     const float nlse2 = rvalid ? -lse[(long long)bh * N + row] * LOG2E : -INFINITY;
     const float Dr = rvalid ? dvec[(long long)bh * N + row] : 0.f;
     const uint64_t scale2 = f2_pack(scale_log2, scale_log2), nlse2x2 = f2_pack(nlse2, nlse2),
@@ -586,49 +597,35 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_cons
         ok = false;
         break;
       }
-      // this dS buffer was read by the dQ product of tile t-2
-      if (t >= 2 && !wait_warp(&sm.ds_empty[b], ((t - 2) >> 1) & 1, wc)) {
-        ok = false;
-        break;
-      }
       tc_fence_after();
       const int kv_valid = t == n - 1 ? last_valid : 64;
+      const int c0 = h * 32;
+      uint32_t sa[32], pa[32];
+      tmem_ld32(tl + T_S + b * 64 + c0, sa);
+      tmem_ld32(tl + T_DP + b * 64 + c0, pa);
+      tmem_wait_ld();
+      uint32_t dh[16], dl[16];
 #pragma unroll
-      for (int sub = 0; sub < 2; ++sub) {
-        const int c0 = h * 32 + sub * 16;
-        uint32_t sa[16], pa[16];
-        tmem_ld16(tl + T_S + b * 64 + c0, sa);
-        tmem_ld16(tl + T_DP + b * 64 + c0, pa);
-        tmem_wait_ld();
-        uint32_t dh[8], dl[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sa[2 * e]), __uint_as_float(sa[2 * e + 1])), scale2,
-                                     nlse2x2);
-          float x0, x1;
-          f2_unpack(x2, x0, x1);
-          float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-          if (kv_valid < 64) {
-            if (c0 + 2 * e >= kv_valid) p0 = 0.f;
-            if (c0 + 2 * e + 1 >= kv_valid) p1 = 0.f;
-          }
-          const uint64_t ds2 = f2_mul(f2_pack(p0, p1),
-                                      f2_sub(f2_pack(__uint_as_float(pa[2 * e]), __uint_as_float(pa[2 * e + 1])), d2));
-          float s0, s1;
-          f2_unpack(ds2, s0, s1);
-          split_bf16(s0, s1, dh[e], dl[e]);
+      for (int e = 0; e < 16; ++e) {
+        const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sa[2 * e]), __uint_as_float(sa[2 * e + 1])), scale2,
+                                   nlse2x2);
+        float x0, x1;
+        f2_unpack(x2, x0, x1);
+        float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+        if (kv_valid < 64) {
+          if (c0 + 2 * e >= kv_valid) p0 = 0.f;
+          if (c0 + 2 * e + 1 >= kv_valid) p1 = 0.f;
         }
-        const uint32_t u0 = c0 >> 3;
-#pragma unroll
-        for (int w = 0; w < 2; ++w) {
-          const uint32_t off = sw128_offset(r, u0 + w);
-          *reinterpret_cast<uint4*>(sm.ds[b][0] + off) =
-              make_uint4(dh[4 * w], dh[4 * w + 1], dh[4 * w + 2], dh[4 * w + 3]);
-          *reinterpret_cast<uint4*>(sm.ds[b][1] + off) =
-              make_uint4(dl[4 * w], dl[4 * w + 1], dl[4 * w + 2], dl[4 * w + 3]);
-        }
+        const uint64_t ds2 = f2_mul(f2_pack(p0, p1),
+                                    f2_sub(f2_pack(__uint_as_float(pa[2 * e]), __uint_as_float(pa[2 * e + 1])), d2));
+        float s0, s1;
+        f2_unpack(ds2, s0, s1);
+        split_bf16(s0, s1, dh[e], dl[e]);
       }
-      fence_proxy_async_smem();
+      // dS hi / lo over this half's own S columns (already read)
+      tmem_st16(tl + T_S + b * 64 + c0, dh);
+      tmem_st16(tl + T_S + b * 64 + c0 + 16, dl);
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sm.ds_full[b]);
     }
@@ -745,8 +742,9 @@ static cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
     e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     bwd_dq_kernel<D><<<dim3(a.Tm, a.BH), DQ_THREADS, smem, s>>>(
-        *a.tm_q, *a.tm_k, *a.tm_v, *a.tm_do, a.lse, a.dvec, a.row_cnt, a.row_idx, a.dq, a.grad_f32, a.N, a.Tm,
-        a.Tn, a.scale, a.scale_log2, a.status, a.wait_limit_ns);
+        *a.tm_k, *a.tm_v, static_cast<const __nv_bfloat16*>(a.q), static_cast<const __half*>(a.do16), a.lse,
+        a.dvec, a.row_cnt, a.row_idx, a.dq, a.grad_f32, a.N, a.Tm, a.Tn, a.scale, a.scale_log2, a.status,
+        a.wait_limit_ns);
     e = cudaGetLastError();
   }
   return e;

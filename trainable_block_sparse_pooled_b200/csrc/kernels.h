@@ -49,6 +49,7 @@ struct BwdArgs {
   const CUtensorMap* tm_k;    // K bf16, box {64, 64, 1}
   const CUtensorMap* tm_v;    // fp16 copy of V, box {64, 64, 1}
   const CUtensorMap* tm_do;   // fp16 copy of dO, box {64, 128, 1}
+  const void* q;
   const void* o;
   const void* o_lo;   // may be null
   const void* dout;
