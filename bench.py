@@ -460,6 +460,75 @@ def run_gpu(args, wl, name):
     return 0
 
 
+def run_sweep(args):
+    """Sparsity sweep on the 1.3B layer shape (B1 H12 d128, smoothed-field inputs):
+    block sparsity 80 / 90 / 95 / 97% (k = (1 - target) / 2, p calibrated) and the
+    k = 100% pass, at N in {8192, 32760, 65536}. One JSON line per point: mask,
+    forward and backward times (CUDA events, median of --steps after --warmup),
+    sparse and dense-equivalent TFLOP/s, and speedup over the k = 100% pass."""
+    import torch
+    from trainable_block_sparse_pooled_b200 import binding as b
+    from trainable_block_sparse_pooled_b200 import calibrate, synth
+    torch.cuda.set_device(0)
+    B, H, d = 1, 12, 128
+    pk, _ = peaks()
+
+    def med_ms(fn):
+        for _ in range(args.warmup):
+            fn()
+        ts = []
+        for _ in range(args.steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return sorted(ts)[len(ts) // 2]
+
+    for N in (8192, 32760, 65536):
+        q, k, v = synth.smoothed_field(B=B, H=H, N=N, d=d, seed=11, device="cuda")
+        dout = synth.normal_like(q.shape, seed=12, device="cuda")
+        s = b.Spa2(B, H, N, d)
+        mask = s.new_mask()
+        o, o_lo = torch.empty_like(q), torch.empty_like(q)
+        lse = torch.empty(B, H, N, dtype=torch.float32, device="cuda")
+        dq, dk, dv = (torch.empty(q.shape, dtype=torch.float32, device="cuda") for _ in range(3))
+        total = B * H * s.Tm * s.Tn
+        dense_flops = 4.0 * B * H * N * N * d
+
+        def kept(kf, pf):
+            s.block_mask(q, k, kf, pf, mask)
+            return mask.kept_blocks()
+
+        points, dense_ms = [], None
+        for target in (None, 0.80, 0.90, 0.95, 0.97):
+            if target is None:
+                kf, pf = 1.0, 0.0
+                sparsity = 1.0 - kept(kf, pf) / total
+            else:
+                kf, pf, sparsity = calibrate.calibrate_p(kept, total, target)
+            s.block_mask(q, k, kf, pf, mask)
+            flops = kept_flops(mask, N, d)
+            mask_ms = med_ms(lambda: s.block_mask(q, k, kf, pf, mask))
+            fwd_ms = med_ms(lambda: s.fwd(q, k, v, mask, o=o, lse=lse, o_lo=o_lo))
+            bwd_ms = med_ms(lambda: s.bwd(q, k, v, o, lse, dout, mask, dq=dq, dk=dk, dv=dv, o_lo=o_lo))
+            s.check()
+            if target is None:
+                dense_ms = (fwd_ms, bwd_ms)
+            line = {"sweep": "sparsity", "N": N, "target_sparsity": target, "block_sparsity": sparsity,
+                    "k_frac": kf, "p_frac": pf, "mask_us": mask_ms * 1e3, "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+                    "fwd_tflops": flops / (fwd_ms * 1e-3) / 1e12, "bwd_tflops": 2.5 * flops / (bwd_ms * 1e-3) / 1e12,
+                    "fwd_frac_burst": flops / (fwd_ms * 1e-3) / 1e12 / pk["bf16_tflops"],
+                    "fwd_dense_equiv_tflops": dense_flops / (fwd_ms * 1e-3) / 1e12,
+                    "speedup_fwd": dense_ms[0] / fwd_ms, "speedup_fwd_bwd": sum(dense_ms) / (fwd_ms + bwd_ms),
+                    "steps": args.steps, "warmup": args.warmup}
+            print(json.dumps(line), flush=True)
+        del q, k, v, dout, s, mask, o, o_lo, lse, dq, dk, dv
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -472,11 +541,15 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the k = 100%% comparison pass")
+    ap.add_argument("--sweep", action="store_true",
+                    help="sparsity sweep (80/90/95/97%% and k = 100%%) at N = 8192, 32760, 65536: one JSON line per point")
     ap.add_argument("--heads", type=int, default=0,
                     help="override the workload's head count (a smaller case of the same layer, for profiling)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.sweep:
+        return run_sweep(args)
     wl = dict(WORKLOADS[args.workload])
     name = args.workload
     if args.heads > 0:

@@ -182,3 +182,56 @@ def test_wan13b_bwd_sampled_blocks():
             acc["dV"].add(dv[0, h, j * 64:j * 64 + gv.shape[0]], gv)
     for a in acc.values():
         a.check()
+
+
+@pytest.mark.slow
+def test_wan14b_fwd_bwd_sampled():
+    """14B layer (B1 H40 N75600 d128, smoothed field + 4 sinks, 591 x 1182 blocks) at
+    95% block sparsity (k = 2.5%, p calibrated): O and LSE of 16 seeded q-blocks plus
+    the ragged last one in heads 0, 17 and 39; dQ of 6 q-blocks and dK, dV of 6
+    kv-blocks plus the ragged last one in heads 0 and 39."""
+    from trainable_block_sparse_pooled_b200 import calibrate
+    B, H, N, d = 1, 40, 75600, 128
+    q, k, v = synth.smoothed_field(B=B, H=H, N=N, d=d, seed=5, device="cuda")
+    dout = synth.normal_like(q.shape, seed=6, device="cuda")
+    s = b.Spa2(B, H, N, d)
+    m = s.new_mask()
+
+    def kept(kf, pf):
+        s.block_mask(q, k, kf, pf, m)
+        return m.kept_blocks()
+
+    kf, pf, sp = calibrate.calibrate_p(kept, B * H * s.Tm * s.Tn, 0.95)
+    assert abs(sp - 0.95) <= 0.0025
+    s.block_mask(q, k, kf, pf, m)
+    o, lse = s.fwd(q, k, v, m)
+    grads = s.bwd(q, k, v, o, lse, dout, m)
+    s.check()
+    heads = [0, 17, 39]
+    dense_all = csr_to_dense(m.row_cnt.cpu().numpy(), m.row_idx.cpu().numpy(), s.Tn)
+    dense = dense_all[:, heads]
+    sl = lambda t: f64(t[:, heads])  # noqa: E731
+    qf, kf_, vf, df = sl(q), sl(k), sl(v), sl(dout)
+    o32 = f64(o[:, heads]) + f64(s.o_lo[:, heads])
+    l64 = lse[:, heads].cpu().numpy()
+    dq, dk, dv = (sl(g) for g in grads)
+    rng = np.random.default_rng(7)
+    acc = {n: Accum(n) for n in ("O (o + o_lo)", "LSE", "dQ", "dK", "dV")}
+    for hi, h in enumerate(heads):
+        blocks = sorted(set(rng.integers(0, s.Tm - 1, 16).tolist()) | {s.Tm - 1})
+        ref = oracle.masked_attn_fwd_rows(qf, kf_, vf, dense, 128, 64, 1 / np.sqrt(d), 0, hi, blocks)
+        for i, (Oi, Li) in ref.items():
+            rows = slice(i * 128, i * 128 + Oi.shape[0])
+            acc["O (o + o_lo)"].add(o32[0, hi, rows], Oi)
+            acc["LSE"].add(l64[0, hi, rows], Li)
+        if h in (0, 39):
+            qb = sorted(set(rng.integers(0, s.Tm, 6).tolist()))
+            kb = sorted(set(rng.integers(0, s.Tn - 1, 6).tolist()) | {s.Tn - 1})
+            sq, skv = oracle.masked_attn_bwd_blocks(qf, kf_, vf, dense, df, 128, 64, 1 / np.sqrt(d), 0, hi, qb, kb)
+            for i, g in sq.items():
+                acc["dQ"].add(dq[0, hi, i * 128:i * 128 + g.shape[0]], g)
+            for j, (gk, gv) in skv.items():
+                acc["dK"].add(dk[0, hi, j * 64:j * 64 + gk.shape[0]], gk)
+                acc["dV"].add(dv[0, hi, j * 64:j * 64 + gv.shape[0]], gv)
+    for a in acc.values():
+        a.check()

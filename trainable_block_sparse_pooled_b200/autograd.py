@@ -1,0 +1,63 @@
+"""`torch.autograd` front end of the sparse attention path.
+
+sparse_attention(q, k, v, k_frac, p_frac) builds the hybrid Top-k + Top-p block
+mask of (q, k) (paper.rainbus.top summary, 方法步骤详情 steps 1-3), runs the
+block-sparse forward (step 4) and, when a gradient is requested, the backward
+through the same mask, which the method holds constant (its trainable part is
+the attention itself: chatpaper.ai abstract (ii)). Every step runs in the
+libspa2 kernels; this module only marshals arguments through the C ABI
+(`binding.Spa2`) and caches the per-shape workspaces.
+"""
+
+from __future__ import annotations
+
+import torch
+
+from . import binding as b
+
+_cache: dict = {}
+
+
+def _spa(B, H, N, d, device) -> b.Spa2:
+    key = (B, H, N, d, str(device))
+    s = _cache.get(key)
+    if s is None:
+        s = _cache[key] = b.Spa2(B, H, N, d, device=device)
+    return s
+
+
+class SparseAttentionFunction(torch.autograd.Function):
+    """O = block-sparse attention of (q, k, v) under the hybrid mask of (q, k).
+
+    q, k, v: [B, H, N, d] bf16 CUDA tensors (d in {64, 128}); gradients come back
+    in bf16. The mask of the last call is kept on the function's context (and
+    returned by `sparse_attention(..., return_mask=True)`).
+    """
+
+    @staticmethod
+    def forward(ctx, q, k, v, k_frac: float, p_frac: float, scale: float = 0.0):
+        if q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16 or v.dtype != torch.bfloat16:
+            raise TypeError("sparse_attention expects bf16 q, k, v")
+        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        B, H, N, d = q.shape
+        s = _spa(B, H, N, d, q.device)
+        mask = s.block_mask(q, k, k_frac, p_frac)
+        o, lse = s.fwd(q, k, v, mask, scale)
+        ctx.save_for_backward(q, k, v, o, lse, s.o_lo)
+        ctx.mask, ctx.scale, ctx.spa = mask, scale, s
+        ctx.mark_non_differentiable(mask.row_cnt)
+        return o, mask.row_cnt  # the kept-block counts, so callers can see the mask
+
+    @staticmethod
+    def backward(ctx, do, _row_cnt_grad):
+        q, k, v, o, lse, o_lo = ctx.saved_tensors
+        dq, dk, dv = ctx.spa.bwd(q, k, v, o, lse, do.contiguous(), ctx.mask, ctx.scale, o_lo=o_lo,
+                                 grad_dtype=b.DTYPE_BF16)
+        ctx.spa.check()  # device-side errors of the mask, forward and backward of this call
+        return dq, dk, dv, None, None, None
+
+
+def sparse_attention(q, k, v, k_frac: float, p_frac: float, scale: float = 0.0, return_mask: bool = False):
+    """Differentiable hybrid block-sparse attention (b_q = 128, b_kv = 64)."""
+    o, row_cnt = SparseAttentionFunction.apply(q, k, v, k_frac, p_frac, scale)
+    return (o, row_cnt) if return_mask else o
