@@ -198,12 +198,15 @@ SPA2_API spa2_status spa2_sparse_attn_fwd(const void* q, const void* k, const vo
  *   dS_ij = P_ij * (dP_ij - D_i),  dQ_i = sum_j dS_ij K_j * scale,
  *   dK_j = sum_i dS_ij^T Q_i * scale.
  * The mask is held constant (no gradient through pooling or selection).
- * Precision: P enters dV = P^T dO as fp16 (P in [0, 1], 11-bit significand)
- * against an fp16 copy of dO; dP = dO V^T takes fp16 copies of dO and V; dS
- * enters dK and dQ as a hi + lo pair of bf16 values (about 16 significant
- * bits); S = Q K^T takes the bf16 inputs; accumulation is fp32 throughout and
- * D uses o + o_lo when o_lo is given. dO or V of magnitude > 65504 is clamped
- * for the fp16 copies and reported as SPA2_ERR_RANGE.
+ * Precision: the dK/dV pass runs every product on fp16 copies of Q, K, V and
+ * dO (bf16 -> fp16 is exact for magnitudes in [2^-14, 65504]; smaller ones
+ * round to fp16 subnormals, absolute error <= 2^-25): S = Q K^T, dP = dO V^T,
+ * and P (in [0, 1]) and dS enter dV = P^T dO and dK = dS^T Q as fp16. The dQ
+ * pass recomputes S from the bf16 inputs and dP from the fp16 copies, and dS
+ * enters dQ = dS K as a hi + lo pair of bf16 values (about 16 significant
+ * bits). Accumulation is fp32 throughout and D uses o + o_lo when o_lo is
+ * given. Q, K, V or dO of magnitude > 65504 is clamped for the fp16 copies
+ * and reported as SPA2_ERR_RANGE.
  * dK and dV are accumulated per kv-block (CSC column), dQ per q-block (CSR
  * row, recomputing S and dP), so no output is accumulated atomically and the
  * results are deterministic.
@@ -216,7 +219,7 @@ SPA2_API spa2_status spa2_sparse_attn_fwd(const void* q, const void* k, const vo
  *   dq, dk, dv       : [B, H, N, d] device outputs of type grad_dtype
  *   grad_dtype       : SPA2_DTYPE_BF16 or SPA2_DTYPE_F32
  *   ws               : spa2_workspace_bytes(SPA2_OP_BWD, ...) bytes (holds D
- *                      and the fp16 copies of dO and V)
+ *                      and the fp16 copies of dO, V, Q and K)
  */
 SPA2_API spa2_status spa2_sparse_attn_bwd(const void* q, const void* k, const void* v, const void* o,
                                           const void* o_lo, const float* lse, const void* dout, int B, int H, int N,

@@ -72,6 +72,8 @@ struct BwdWs {
   float* dvec;
   void* do16;
   void* v16;
+  void* q16;
+  void* k16;
   size_t bytes;
 };
 static BwdWs bwd_ws(void* ws, const Shape& s) {
@@ -84,6 +86,10 @@ static BwdWs bwd_ws(void* ws, const Shape& s) {
   w.do16 = base + off;
   off += al256((size_t)s.BH * s.N * s.d * 2);
   w.v16 = base + off;
+  off += al256((size_t)s.BH * s.N * s.d * 2);
+  w.q16 = base + off;
+  off += al256((size_t)s.BH * s.N * s.d * 2);
+  w.k16 = base + off;
   off += al256((size_t)s.BH * s.N * s.d * 2);
   w.bytes = off;
   return w;
@@ -291,13 +297,14 @@ spa2_status spa2_sparse_attn_bwd(const void* q, const void* k, const void* v, co
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)d);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const bool f32 = grad_dtype == SPA2_DTYPE_F32;
-  CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tq, tk, tv, tdo, tq16, tk16;
   if (!make_map(&tq, q, s, 128) || !make_map(&tk, k, s, 64) || !make_map(&tv, w.v16, s, 64, true) ||
-      !make_map(&tdo, w.do16, s, 128, true))
+      !make_map(&tdo, w.do16, s, 128, true) || !make_map(&tq16, w.q16, s, 128, true) ||
+      !make_map(&tk16, w.k16, s, 64, true))
     return SPA2_ERR_CUDA;
   SPA2_CUDA_TRY(cudaMemsetAsync(w.status, 0, 4, st));
-  BwdArgs a{&tq, &tk, &tv, &tdo, q, o, o_lo, dout, v, lse, mask->row_cnt, mask->row_idx, mask->col_cnt,
-            mask->col_idx, w.dvec, w.do16, w.v16, dq, dk, dv, f32 ? 1 : 0, (int)s.BH, s.N, s.Tm, s.Tn, scale,
+  BwdArgs a{&tq, &tk, &tv, &tdo, &tq16, &tk16, q, k, o, o_lo, dout, v, lse, mask->row_cnt, mask->row_idx, mask->col_cnt,
+            mask->col_idx, w.dvec, w.do16, w.v16, w.q16, w.k16, dq, dk, dv, f32 ? 1 : 0, (int)s.BH, s.N, s.Tm, s.Tn, scale,
             scale * 1.4426950408889634f, w.status, g_wait_limit_ns};
   SPA2_CUDA_TRY(launch_bwd(a, d, st));
   return SPA2_OK;

@@ -5,25 +5,27 @@
 //   dV_j += P^T dO_i      dP = dO_i V_j^T      dS = P * (dP - D_i)
 //   dQ_i += dS K_j * sc   dK_j += dS^T Q_i * sc,  D_i = rowsum(dO_i * O_i).
 //
-// bwd_pre_kernel   D = rowsum(dO * (O + O_lo)) in fp32, and fp16 copies of dO
-//                  and V for the fp16 products below (|x| > 65504 is clamped
+// bwd_pre_kernel   D = rowsum(dO * (O + O_lo)) in fp32, and fp16 copies of dO,
+//                  V, Q and K for the fp16 products below (|x| > 65504 is clamped
 //                  and reported as SPA2_ERR_RANGE).
 // bwd_dkdv_kernel  one CTA per (kv-block j, head), looping over the q-blocks i
 //                  that keep j (CSC column of j), accumulating dV_j and dK_j in
 //                  TMEM (tcgen05 MMAs, fp32 accumulation):
-//                    S   = Q_i K_j^T    bf16  M=128 (q) N=64 (kv) K=d    A,B K-major
+//                    S   = Q_i K_j^T    fp16  M=128 (q) N=64 (kv) K=d    A,B K-major
 //                    dP  = dO_i V_j^T   fp16  M=128 (q) N=64 (kv) K=d    A,B K-major
 //                    dV^T += dO_i^T P   fp16  M=d       N=64 (kv) K=128  A,B MN-major
-//                    dK^T += Q_i^T dS   bf16  M=d       N=64 (kv) K=128  A,B MN-major
-//                  Warps 0-7 turn S, dP into P (fp16: 11-bit significand, P in
-//                  [0, 1]) and dS (a hi + lo pair of bf16 tiles, about 16
-//                  significant bits, since a bf16 rounding of dS is amplified by
-//                  large keys in dK and dQ); warpgroup h handles kv columns
-//                  32h .. 32h+31, thread = query row. The dK^T product runs once
-//                  per half of dS. Warp 8: TMA producer; warp 9: MMA issuer.
+//                    dK^T += Q_i^T dS   fp16  M=d       N=64 (kv) K=128  A,B MN-major
+//                  (fp16 copies of Q, K, V, dO). Warps 0-7 turn S, dP into P and
+//                  dS as fp16 tiles (11-bit significands; an fp16 dS keeps dK
+//                  within a few 1e-3 of the float64 result on the sink-key cases,
+//                  where a bf16 dS does not); warpgroup h handles kv columns
+//                  32h .. 32h+31, thread = query row. Warp 8: TMA producer; warp 9:
+//                  MMA issuer.
 // bwd_dq_kernel    one CTA per (q-block i, head), looping over the kv-blocks j
-//                  that i keeps (CSR row of i); recomputes S and dP, forms dS as
-//                  above and accumulates dQ_i = sum_j dS_ij K_j in TMEM
+//                  that i keeps (CSR row of i); recomputes S and dP, forms dS as a
+//                  hi + lo pair of bf16 values (about 16 significant bits: dQ is
+//                  the gradient most sensitive to dS rounding) and accumulates
+//                  dQ_i = sum_j dS_ij K_j in TMEM
 //                    dQ  += dS K_j      bf16  M=128 (q) N=d       K=64   A K-, B MN-major
 //                  then writes it once: no atomics and no fp32 scratch for dQ.
 //                  For d = 64 the dV^T / dK^T MMAs still run at M = 128 (the
@@ -45,12 +47,12 @@ constexpr int BWD_THREADS = 320;  // P/dS x 8 warps, TMA, MMA
 template <int D>
 struct BwdSmem {
   static constexpr int CH = D / 64;
-  alignas(1024) uint8_t k[CH][64 * 128];         // K_j bf16
+  alignas(1024) uint8_t k[CH][64 * 128];         // K_j fp16
   alignas(1024) uint8_t v[CH][64 * 128];         // V_j fp16
-  alignas(1024) uint8_t q[2][CH][128 * 128];     // Q_i bf16
+  alignas(1024) uint8_t q[2][CH][128 * 128];     // Q_i fp16
   alignas(1024) uint8_t dO[2][CH][128 * 128];    // dO_i fp16
   alignas(1024) uint8_t p[128 * 128];            // P  [128 q][64 kv] fp16
-  alignas(1024) uint8_t ds[2][128 * 128];        // dS [128 q][64 kv]: hi, lo bf16 tiles
+  alignas(1024) uint8_t ds[128 * 128];           // dS [128 q][64 kv] fp16
   uint64_t kv_full;
   uint64_t qd_full[2], qd_empty[2], sdp_full[2];
   uint64_t pds_full, pds_empty, acc_done, drain;
@@ -102,8 +104,8 @@ SPA2_DEV void split_bf16(float a, float b, uint32_t& hi, uint32_t& lo) {
 }  // namespace
 
 template <int D>
-__global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
-                                                                  const __grid_constant__ CUtensorMap tm_k,
+__global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q16,
+                                                                  const __grid_constant__ CUtensorMap tm_k16,
                                                                   const __grid_constant__ CUtensorMap tm_v16,
                                                                   const __grid_constant__ CUtensorMap tm_do16,
                                                                   const float* __restrict__ lse,
@@ -114,10 +116,10 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
                                                              float scale, float scale_log2, int* status,
                                                              unsigned long long wait_limit_ns) {
   constexpr int CH = D / 64;
-  constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, false, false);
-  constexpr uint32_t IDESC_DP = idesc_bf16_f32(128, 64, false, false, /*f16=*/true);
-  constexpr uint32_t IDESC_DV = idesc_bf16_f32(128, 64, true, true, /*f16=*/true);
-  constexpr uint32_t IDESC_T = idesc_bf16_f32(128, 64, true, true);
+  // every product of this kernel takes fp16 operands (fp16 copies of Q, K, V, dO)
+  constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, false, false, /*f16=*/true);
+  constexpr uint32_t IDESC_DP = IDESC_S;
+  constexpr uint32_t IDESC_T = idesc_bf16_f32(128, 64, true, true, /*f16=*/true);  // dV^T and dK^T
   constexpr uint32_t QT_BYTES = 128 * D * 2;
   constexpr uint32_t KV_BYTES = 64 * D * 2;
   // MN-major A operand (dO^T, Q^T): stride between the two 64-row halves of M = d
@@ -171,13 +173,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
   if (warp == 8) {
     // ---------------- TMA producer ----------------
     if (lane == 0 && n > 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_q16);
+      tma_prefetch_desc(&tm_k16);
       tma_prefetch_desc(&tm_v16);
       tma_prefetch_desc(&tm_do16);
       mbar_expect_tx(&sm.kv_full, 2 * KV_BYTES);
       for (int c = 0; c < CH; ++c) {
-        tma_load_3d(sm.k[c], &tm_k, &sm.kv_full, c * 64, j * 64, bh);
+        tma_load_3d(sm.k[c], &tm_k16, &sm.kv_full, c * 64, j * 64, bh);
         tma_load_3d(sm.v[c], &tm_v16, &sm.kv_full, c * 64, j * 64, bh);
       }
       int issued = 0;
@@ -192,7 +194,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
         }
         mbar_expect_tx(&sm.qd_full[s], 2 * QT_BYTES);
         for (int c = 0; c < CH; ++c) {
-          tma_load_3d(sm.q[s][c], &tm_q, &sm.qd_full[s], c * 64, i * 128, bh);
+          tma_load_3d(sm.q[s][c], &tm_q16, &sm.qd_full[s], c * 64, i * 128, bh);
           tma_load_3d(sm.dO[s][c], &tm_do16, &sm.qd_full[s], c * 64, i * 128, bh);
         }
         issued = t + 1;
@@ -203,7 +205,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
   } else if (warp == 9) {
     // ---------------- MMA issuer ----------------
     if (lane == 0 && n > 0) {
-      const uint32_t p_addr = smem_u32(sm.p), ds_addr = smem_u32(sm.ds[0]);
+      const uint32_t p_addr = smem_u32(sm.p), ds_addr = smem_u32(sm.ds);
       // S(t), dP(t) into TMEM buffer t mod 2 (Q / dO stage t mod 2)
       auto issue_sdp = [&](int t) {
         const int s = t & 1;
@@ -239,19 +241,15 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
             break;
           }
           tc_fence_after();
-          // dV^T += dO^T P (fp16); dK^T += Q^T (dS_hi + dS_lo) (bf16); K = 128 query rows
+          // dV^T += dO^T P; dK^T += Q^T dS (fp16); K = 128 query rows
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ss(tmem + T_DV, sdesc_sw128(smem_u32(sm.dO[su][0]) + kk * 2048, LBO_DT, 1024),
-                   sdesc_sw128(p_addr + kk * 2048, 0, 1024), IDESC_DV, (u > 0 || kk > 0) ? 1u : 0u);
+                   sdesc_sw128(p_addr + kk * 2048, 0, 1024), IDESC_T, (u > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
-          for (int part = 0; part < 2; ++part) {
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma_ss(tmem + T_DK, sdesc_sw128(smem_u32(sm.q[su][0]) + kk * 2048, LBO_DT, 1024),
-                     sdesc_sw128(ds_addr + part * (128 * 128) + kk * 2048, 0, 1024), IDESC_T,
-                     (u > 0 || part > 0 || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tmem + T_DK, sdesc_sw128(smem_u32(sm.q[su][0]) + kk * 2048, LBO_DT, 1024),
+                   sdesc_sw128(ds_addr + kk * 2048, 0, 1024), IDESC_T, (u > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&sm.qd_empty[su]);
           mma_commit(&sm.pds_empty);
           if (T == u + 1 && T < n) {
@@ -309,7 +307,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
         tmem_ld16(tl + T_S + s * 64 + c0, sa);
         tmem_ld16(tl + T_DP + s * 64 + c0, pa);
         tmem_wait_ld();
-        uint32_t pk[8], dh[8], dl[8];
+        uint32_t pk[8], dk16[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sa[2 * e]), __uint_as_float(sa[2 * e + 1])), scale2,
@@ -326,17 +324,15 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
                                       f2_sub(f2_pack(__uint_as_float(pa[2 * e]), __uint_as_float(pa[2 * e + 1])), d2));
           float s0, s1;
           f2_unpack(ds2, s0, s1);
-          split_bf16(s0, s1, dh[e], dl[e]);
+          dk16[e] = pack_f16(s0, s1);
         }
         const uint32_t u0 = c0 >> 3;  // 16-byte unit of the slice's first column
 #pragma unroll
         for (int w = 0; w < 2; ++w) {
           const uint32_t off = sw128_offset(r, u0 + w);
           *reinterpret_cast<uint4*>(sm.p + off) = make_uint4(pk[4 * w], pk[4 * w + 1], pk[4 * w + 2], pk[4 * w + 3]);
-          *reinterpret_cast<uint4*>(sm.ds[0] + off) =
-              make_uint4(dh[4 * w], dh[4 * w + 1], dh[4 * w + 2], dh[4 * w + 3]);
-          *reinterpret_cast<uint4*>(sm.ds[1] + off) =
-              make_uint4(dl[4 * w], dl[4 * w + 1], dl[4 * w + 2], dl[4 * w + 3]);
+          *reinterpret_cast<uint4*>(sm.ds + off) =
+              make_uint4(dk16[4 * w], dk16[4 * w + 1], dk16[4 * w + 2], dk16[4 * w + 3]);
         }
       }
       fence_proxy_async_smem();
@@ -669,15 +665,18 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_cons
   }
 }
 
-// D = rowsum(dO * (O + O_lo)) in fp32; fp16 copies of the dO and V rows
+// D = rowsum(dO * (O + O_lo)) in fp32; fp16 copies of the dO, V, Q and K rows
 // (|x| > 65504 clamped and reported). 16 threads per row.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
                                                       const __nv_bfloat16* __restrict__ o_lo,
                                                       const __nv_bfloat16* __restrict__ dout,
                                                       const __nv_bfloat16* __restrict__ v,
-                                                      float* __restrict__ dvec, uint32_t* __restrict__ do16, uint32_t* __restrict__ v16,
-                                                      long long rows, int* status) {
+                                                      const __nv_bfloat16* __restrict__ q,
+                                                      const __nv_bfloat16* __restrict__ k,
+                                                      float* __restrict__ dvec, uint32_t* __restrict__ do16,
+                                                      uint32_t* __restrict__ v16, uint32_t* __restrict__ q16,
+                                                      uint32_t* __restrict__ k16, long long rows, int* status) {
   constexpr int TPR = 16;
   constexpr int EPT = D / TPR;  // 8 (d=128) or 4 (d=64) elements per thread
   const long long row = (long long)blockIdx.x * (256 / TPR) + threadIdx.x / TPR;
@@ -708,6 +707,18 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __res
       }
       do16[(off + e) / 2] = pack_f16(b.x, b.y);
       v16[(off + e) / 2] = pack_f16(w.x, w.y);
+      float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(q + off + e));
+      float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(k + off + e));
+      if (!(fabsf(x.x) <= 65504.f) || !(fabsf(x.y) <= 65504.f) || !(fabsf(y.x) <= 65504.f) ||
+          !(fabsf(y.y) <= 65504.f)) {
+        bad = true;
+        x.x = fminf(fmaxf(x.x, -65504.f), 65504.f);
+        x.y = fminf(fmaxf(x.y, -65504.f), 65504.f);
+        y.x = fminf(fmaxf(y.x, -65504.f), 65504.f);
+        y.y = fminf(fmaxf(y.y, -65504.f), 65504.f);
+      }
+      q16[(off + e) / 2] = pack_f16(x.x, x.y);
+      k16[(off + e) / 2] = pack_f16(y.x, y.y);
     }
   }
 #pragma unroll
@@ -722,7 +733,8 @@ static cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
   // 1. D and the fp16 copies of dO and V
   bwd_pre_kernel<D><<<(unsigned)((rows + 15) / 16), 256, 0, s>>>(
       (const __nv_bfloat16*)a.o, (const __nv_bfloat16*)a.o_lo, (const __nv_bfloat16*)a.dout,
-      (const __nv_bfloat16*)a.v, a.dvec, (uint32_t*)a.do16, (uint32_t*)a.v16, rows, a.status);
+      (const __nv_bfloat16*)a.v, (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, a.dvec, (uint32_t*)a.do16,
+      (uint32_t*)a.v16, (uint32_t*)a.q16, (uint32_t*)a.k16, rows, a.status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // 2. dK, dV (kv-major)
@@ -731,7 +743,7 @@ static cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
     e = cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     bwd_dkdv_kernel<D><<<dim3(a.Tn, a.BH), BWD_THREADS, smem, s>>>(
-        *a.tm_q, *a.tm_k, *a.tm_v, *a.tm_do, a.lse, a.dvec, a.col_cnt, a.col_idx, a.dk, a.dv, a.grad_f32, a.N, a.Tm,
+        *a.tm_q16, *a.tm_k16, *a.tm_v, *a.tm_do, a.lse, a.dvec, a.col_cnt, a.col_idx, a.dk, a.dv, a.grad_f32, a.N, a.Tm,
         a.Tn, a.scale, a.scale_log2, a.status, a.wait_limit_ns);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -49,7 +49,10 @@ struct BwdArgs {
   const CUtensorMap* tm_k;    // K bf16, box {64, 64, 1}
   const CUtensorMap* tm_v;    // fp16 copy of V, box {64, 64, 1}
   const CUtensorMap* tm_do;   // fp16 copy of dO, box {64, 128, 1}
+  const CUtensorMap* tm_q16;  // fp16 copy of Q, box {64, 128, 1}
+  const CUtensorMap* tm_k16;  // fp16 copy of K, box {64, 64, 1}
   const void* q;
+  const void* k;
   const void* o;
   const void* o_lo;   // may be null
   const void* dout;
@@ -62,6 +65,8 @@ struct BwdArgs {
   float* dvec;     // [BH, N]
   void* do16;      // [BH, N, d] fp16
   void* v16;       // [BH, N, d] fp16
+  void* q16;       // [BH, N, d] fp16
+  void* k16;       // [BH, N, d] fp16
   void* dq;
   void* dk;
   void* dv;
