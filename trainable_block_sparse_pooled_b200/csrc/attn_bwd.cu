@@ -51,11 +51,11 @@ struct BwdSmem {
   alignas(1024) uint8_t v[CH][64 * 128];         // V_j fp16
   alignas(1024) uint8_t q[2][CH][128 * 128];     // Q_i fp16
   alignas(1024) uint8_t dO[2][CH][128 * 128];    // dO_i fp16
-  alignas(1024) uint8_t p[128 * 128];            // P  [128 q][64 kv] fp16
-  alignas(1024) uint8_t ds[128 * 128];           // dS [128 q][64 kv] fp16
+  alignas(1024) uint8_t p[2][128 * 128];         // P  [128 q][64 kv] fp16, tile t in buffer t mod 2
+  alignas(1024) uint8_t ds[2][128 * 128];        // dS [128 q][64 kv] fp16
   uint64_t kv_full;
   uint64_t qd_full[2], qd_empty[2], sdp_full[2];
-  uint64_t pds_full, pds_empty, acc_done, drain;
+  uint64_t pds_full[2], pds_empty[2], acc_done, drain;
   uint32_t tmem_base;
   int abort_flag;
   int never;
@@ -130,7 +130,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
   extern __shared__ uint8_t smem_raw[];
   BwdSmem<D>& sm = *reinterpret_cast<BwdSmem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
-  const int warp = threadIdx.x >> 5;
+  const int warp = __shfl_sync(0xffffffffu, (int)(threadIdx.x >> 5), 0);  // warp-uniform
   const uint32_t lane = lane_id();
   const int j = blockIdx.x;
   const int bh = blockIdx.y;
@@ -147,9 +147,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
       mbar_init(&sm.qd_full[s], 1);
       mbar_init(&sm.qd_empty[s], 1);
       mbar_init(&sm.sdp_full[s], 1);
+      mbar_init(&sm.pds_full[s], 256);
+      mbar_init(&sm.pds_empty[s], 1);
     }
-    mbar_init(&sm.pds_full, 256);
-    mbar_init(&sm.pds_empty, 1);
     mbar_init(&sm.acc_done, 1);
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
   const WaitCtx wc{&sm.abort_flag, status, wait_limit_ns};
   const WaitCtx drain_wc{&sm.never, nullptr, wait_limit_ns};
 
-  int n = col_cnt[colid];
+  int n = __shfl_sync(0xffffffffu, col_cnt[colid], 0);  // warp-uniform
   if (n < 0 || n > Tm) {
     if (threadIdx.x == 0) report(status, SPA2_ERR_DEVICE_BOUNDS);
     n = -1;  // error: write nothing
@@ -204,8 +204,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
     }
   } else if (warp == 9) {
     // ---------------- MMA issuer ----------------
-    if (lane == 0 && n > 0) {
-      const uint32_t p_addr = smem_u32(sm.p), ds_addr = smem_u32(sm.ds);
+    if (n > 0) {  // all 32 lanes; elect.sync picks the issuing lane
+      const uint32_t p_addr = smem_u32(sm.p[0]), ds_addr = smem_u32(sm.ds[0]);
       // S(t), dP(t) into TMEM buffer t mod 2 (Q / dO stage t mod 2)
       auto issue_sdp = [&](int t) {
         const int s = t & 1;
@@ -214,56 +214,69 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (64 * 128) + (kk & 3) * 32;
           const uint32_t offq = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-          mma_ss(tmem + T_S + s * 64, sdesc_sw128(smem_u32(sm.q[s][0]) + offq, 16, 1024),
-                 sdesc_sw128(smem_u32(sm.k[0]) + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+          mma_ss_el(tmem + T_S + s * 64, sdesc_sw128(smem_u32(sm.q[s][0]) + offq, 16, 1024),
+                    sdesc_sw128(smem_u32(sm.k[0]) + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (64 * 128) + (kk & 3) * 32;
           const uint32_t offq = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-          mma_ss(tmem + T_DP + s * 64, sdesc_sw128(smem_u32(sm.dO[s][0]) + offq, 16, 1024),
-                 sdesc_sw128(smem_u32(sm.v[0]) + off, 16, 1024), IDESC_DP, kk > 0 ? 1u : 0u);
+          mma_ss_el(tmem + T_DP + s * 64, sdesc_sw128(smem_u32(sm.dO[s][0]) + offq, 16, 1024),
+                    sdesc_sw128(smem_u32(sm.v[0]) + off, 16, 1024), IDESC_DP, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&sm.sdp_full[s]);
+        mma_commit_el(&sm.sdp_full[s]);
       };
-      // S/dP(u+1) goes ahead of dV/dK(u) only when its Q / dO tile has already
-      // landed; a late tile never holds back the products the P / dS warps wait on
-      int T = 0;  // S/dP issued
-      bool ok = wait_bar(&sm.kv_full, 0, wc) && wait_bar(&sm.qd_full[0], 0, wc);
-      if (ok) {
-        issue_sdp(0);
-        T = 1;
-        for (int u = 0; u < n && ok; ++u) {
-          if (T == u + 1 && T < n && mbar_test_wait(&sm.qd_full[T & 1], (T >> 1) & 1)) issue_sdp(T++);
-          const int su = u & 1;
-          if (!wait_bar(&sm.pds_full, u & 1, wc)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          // dV^T += dO^T P; dK^T += Q^T dS (fp16); K = 128 query rows
+      // dV^T += dO^T P; dK^T += Q^T dS (fp16); K = 128 query rows
+      auto issue_dvdk = [&](int u) {
+        const int su = u & 1;
+        const uint32_t pb = (uint32_t)su * (128 * 128);
+        tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tmem + T_DV, sdesc_sw128(smem_u32(sm.dO[su][0]) + kk * 2048, LBO_DT, 1024),
-                   sdesc_sw128(p_addr + kk * 2048, 0, 1024), IDESC_T, (u > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss_el(tmem + T_DV, sdesc_sw128(smem_u32(sm.dO[su][0]) + kk * 2048, LBO_DT, 1024),
+                    sdesc_sw128(p_addr + pb + kk * 2048, 0, 1024), IDESC_T, (u > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tmem + T_DK, sdesc_sw128(smem_u32(sm.q[su][0]) + kk * 2048, LBO_DT, 1024),
-                   sdesc_sw128(ds_addr + kk * 2048, 0, 1024), IDESC_T, (u > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&sm.qd_empty[su]);
-          mma_commit(&sm.pds_empty);
-          if (T == u + 1 && T < n) {
-            if (!wait_bar(&sm.qd_full[T & 1], (T >> 1) & 1, wc)) {
-              ok = false;
-              break;
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss_el(tmem + T_DK, sdesc_sw128(smem_u32(sm.q[su][0]) + kk * 2048, LBO_DT, 1024),
+                    sdesc_sw128(ds_addr + pb + kk * 2048, 0, 1024), IDESC_T, (u > 0 || kk > 0) ? 1u : 0u);
+        mma_commit_el(&sm.qd_empty[su]);
+        mma_commit_el(&sm.pds_empty[su]);
+      };
+      // Issue whichever product is ready. S/dP(T) needs its Q / dO tile and
+      // dV/dK(T-2) issued (the P / dS warps are then done reading TMEM buffer
+      // T mod 2); dV/dK(U) needs the P / dS tile of U. Of two ready products
+      // S/dP goes first, so the P / dS warps work on tile U+1 while the tensor
+      // pipe runs dV/dK(U).
+      int T = 0, U = 0;  // S/dP and dV/dK products issued
+      bool ok = wait_bar_all(&sm.kv_full, 0, wc);
+      uint64_t t0 = 0;
+      uint32_t idle = 0;
+      while (ok && U < n) {
+        if (T < n && T <= U + 1 && test_wait_all(&sm.qd_full[T & 1], (T >> 1) & 1)) {
+          issue_sdp(T++);
+          idle = 0;
+          t0 = 0;
+        } else if (U < T && test_wait_all(&sm.pds_full[U & 1], (U >> 1) & 1)) {
+          issue_dvdk(U++);
+          idle = 0;
+          t0 = 0;
+        } else if ((++idle & 63u) == 0u) {
+          // the lanes agree on giving up (abort raised elsewhere, or the time limit)
+          const uint64_t now = globaltimer_ns();
+          if (t0 == 0) t0 = now;
+          const bool aborted = __any_sync(0xffffffffu, *wc.abort_flag != 0);
+          if (aborted || __any_sync(0xffffffffu, now - t0 > wait_limit_ns)) {
+            if (!aborted) {
+              report(status, SPA2_ERR_DEVICE_TIMEOUT);
+              *wc.abort_flag = 1;
             }
-            issue_sdp(T++);
+            ok = false;
           }
         }
-        if (ok) mma_commit(&sm.acc_done);
       }
-      mma_commit(&sm.drain);
-      wait_bar(&sm.drain, 0, drain_wc);
+      if (ok) mma_commit_el(&sm.acc_done);
+      mma_commit_el(&sm.drain);
+      wait_bar_all(&sm.drain, 0, drain_wc);
     }
   } else {
     // ---------------- P / dS warps 0-7 ----------------
@@ -294,8 +307,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
         break;
       }
       tc_fence_after();
-      // the P / dS tiles of the previous tile must have been consumed
-      if (t >= 1 && !wait_warp(&sm.pds_empty, (t - 1) & 1, wc)) {
+      // P / dS buffer t mod 2 must have been consumed by dV/dK(t-2)
+      if (t >= 2 && !wait_warp(&sm.pds_empty[s], ((t >> 1) - 1) & 1, wc)) {
         ok = false;
         break;
       }
@@ -330,14 +343,15 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
 #pragma unroll
         for (int w = 0; w < 2; ++w) {
           const uint32_t off = sw128_offset(r, u0 + w);
-          *reinterpret_cast<uint4*>(sm.p + off) = make_uint4(pk[4 * w], pk[4 * w + 1], pk[4 * w + 2], pk[4 * w + 3]);
-          *reinterpret_cast<uint4*>(sm.ds + off) =
+          *reinterpret_cast<uint4*>(sm.p[s] + off) =
+              make_uint4(pk[4 * w], pk[4 * w + 1], pk[4 * w + 2], pk[4 * w + 3]);
+          *reinterpret_cast<uint4*>(sm.ds[s] + off) =
               make_uint4(dk16[4 * w], dk16[4 * w + 1], dk16[4 * w + 2], dk16[4 * w + 3]);
         }
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&sm.pds_full);
+      mbar_arrive(&sm.pds_full[s]);
     }
     // epilogue: warpgroup 0 writes dV_j = (dV^T)^T, warpgroup 1 dK_j = scale * (dK^T)^T;
     // thread r <-> feature r
@@ -443,7 +457,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_cons
   extern __shared__ uint8_t smem_raw[];
   DqSmem<D>& sm = *reinterpret_cast<DqSmem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
-  const int warp = threadIdx.x >> 5;
+  const int warp = __shfl_sync(0xffffffffu, (int)(threadIdx.x >> 5), 0);  // warp-uniform
   const uint32_t lane = lane_id();
   const int i = blockIdx.x;
   const int bh = blockIdx.y;
@@ -476,7 +490,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_cons
   const WaitCtx wc{&sm.abort_flag, status, wait_limit_ns};
   const WaitCtx drain_wc{&sm.never, nullptr, wait_limit_ns};
 
-  int n = row_cnt[rowid];
+  int n = __shfl_sync(0xffffffffu, row_cnt[rowid], 0);  // warp-uniform
   if (n < 1 || n > Tn) {
     if (threadIdx.x == 0) report(status, SPA2_ERR_DEVICE_BOUNDS);
     n = 0;
@@ -510,47 +524,47 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_cons
     }
   } else if (warp == 9) {
     // ---------------- MMA issuer: S(t), dP(t), then dQ += dS(t-1) K(t-1), all TS ----------------
-    if (lane == 0 && n > 0) {
-      if (wait_bar(&sm.qd_ready, 0, wc)) {
+    if (n > 0) {  // all 32 lanes; elect.sync picks the issuing lane
+      if (wait_bar_all(&sm.qd_ready, 0, wc)) {
         for (int t = 0; t <= n; ++t) {
           if (t < n) {
             const int b = t & 1, slot = t % DQ_KS;
-            if (!wait_bar(&sm.kv_full[slot], (t / DQ_KS) & 1, wc)) break;
+            if (!wait_bar_all(&sm.kv_full[slot], (t / DQ_KS) & 1, wc)) break;
             tc_fence_after();
             const uint32_t kb = smem_u32(sm.k[slot][0]), vb = smem_u32(sm.v[slot][0]);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t off = (kk >> 2) * (64 * 128) + (kk & 3) * 32;
-              mma_ts(tmem + T_S + b * 64, tmem + T_Q + kk * 8, sdesc_sw128(kb + off, 16, 1024), IDESC_S,
-                     kk > 0 ? 1u : 0u);
+              mma_ts_el(tmem + T_S + b * 64, tmem + T_Q + kk * 8, sdesc_sw128(kb + off, 16, 1024), IDESC_S,
+                        kk > 0 ? 1u : 0u);
             }
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t off = (kk >> 2) * (64 * 128) + (kk & 3) * 32;
-              mma_ts(tmem + T_DP + b * 64, tmem + T_DO + kk * 8, sdesc_sw128(vb + off, 16, 1024), IDESC_DP,
-                     kk > 0 ? 1u : 0u);
+              mma_ts_el(tmem + T_DP + b * 64, tmem + T_DO + kk * 8, sdesc_sw128(vb + off, 16, 1024), IDESC_DP,
+                        kk > 0 ? 1u : 0u);
             }
-            mma_commit(&sm.sdp_full[b]);
+            mma_commit_el(&sm.sdp_full[b]);
           }
           if (t >= 1) {
             const int u = t - 1, b = u & 1, slot = u % DQ_KS;
-            if (!wait_bar(&sm.ds_full[b], (u >> 1) & 1, wc)) break;
+            if (!wait_bar_all(&sm.ds_full[b], (u >> 1) & 1, wc)) break;
             tc_fence_after();
             const uint32_t kb = smem_u32(sm.k[slot][0]);
 #pragma unroll
             for (int part = 0; part < 2; ++part) {
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
-                mma_ts(tmem + T_DQ, tmem + T_S + b * 64 + (kk >> 1) * 32 + part * 16 + (kk & 1) * 8,
-                       sdesc_sw128(kb + kk * 2048, 64 * 128, 1024), IDESC_Q, (u > 0 || part > 0 || kk > 0) ? 1u : 0u);
+                mma_ts_el(tmem + T_DQ, tmem + T_S + b * 64 + (kk >> 1) * 32 + part * 16 + (kk & 1) * 8,
+                          sdesc_sw128(kb + kk * 2048, 64 * 128, 1024), IDESC_Q, (u > 0 || part > 0 || kk > 0) ? 1u : 0u);
             }
-            mma_commit(&sm.kv_empty[slot]);
+            mma_commit_el(&sm.kv_empty[slot]);
           }
         }
-        mma_commit(&sm.acc_done);
+        mma_commit_el(&sm.acc_done);
       }
-      mma_commit(&sm.drain);
-      wait_bar(&sm.drain, 0, drain_wc);
+      mma_commit_el(&sm.drain);
+      wait_bar_all(&sm.drain, 0, drain_wc);
     }
   } else {
     // ---------------- dS warps 0-7: warpgroup h handles kv columns 32h .. 32h+31 ----------------

@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(192, 2) fwd_kernel(const __grid_constant__ CUt
   extern __shared__ uint8_t smem_raw[];
   FwdSmem<D>& sm = *reinterpret_cast<FwdSmem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
-  const int warp = threadIdx.x >> 5;
+  const int warp = __shfl_sync(0xffffffffu, (int)(threadIdx.x >> 5), 0);  // warp-uniform
   const uint32_t lane = lane_id();
   const int i = blockIdx.x;
   const int bh = blockIdx.y;
@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(192, 2) fwd_kernel(const __grid_constant__ CUt
   const uint32_t tmem = sm.tmem_base;
   const WaitCtx wc{&sm.abort_flag, status, wait_limit_ns};
 
-  int n = row_cnt[rowid];
+  int n = __shfl_sync(0xffffffffu, row_cnt[rowid], 0);  // warp-uniform
   if (n < 1 || n > Tn) {
     if (threadIdx.x == 0) report(status, SPA2_ERR_DEVICE_BOUNDS);
     n = 0;
@@ -143,41 +143,41 @@ __global__ void __launch_bounds__(192, 2) fwd_kernel(const __grid_constant__ CUt
     }
   } else if (warp == 5) {
     // ---------------- MMA issuer ----------------
-    if (lane == 0 && n > 0) {
+    if (n > 0) {  // all 32 lanes; elect.sync picks the issuing lane
       const uint32_t tmem_o = tmem + 128;
-      if (wait_bar(&sm.q_full, 0, wc)) {
+      if (wait_bar_all(&sm.q_full, 0, wc)) {
         for (int t = 0; t <= n; ++t) {
           if (t < n) {
             const int s = t & 1;
-            if (!wait_bar(&sm.k_full[s], (t >> 1) & 1, wc)) break;
+            if (!wait_bar_all(&sm.k_full[s], (t >> 1) & 1, wc)) break;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint64_t a = sdesc_sw128(smem_u32(sm.q[kk >> 2]) + (kk & 3) * 32, 16, 1024);
               const uint64_t b = sdesc_sw128(smem_u32(sm.k[s][kk >> 2]) + (kk & 3) * 32, 16, 1024);
-              mma_ss(tmem + s * 64, a, b, IDESC_S, kk > 0 ? 1u : 0u);
+              mma_ss_el(tmem + s * 64, a, b, IDESC_S, kk > 0 ? 1u : 0u);
             }
-            mma_commit(&sm.s_full[s]);
+            mma_commit_el(&sm.s_full[s]);
           }
           if (t >= 1) {
             const int u = t - 1, su = u & 1;
-            if (!wait_bar(&sm.p_full[su], (u >> 1) & 1, wc)) break;
-            if (!wait_bar(&sm.v_full[su], (u >> 1) & 1, wc)) break;
+            if (!wait_bar_all(&sm.p_full[su], (u >> 1) & 1, wc)) break;
+            if (!wait_bar_all(&sm.v_full[su], (u >> 1) & 1, wc)) break;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint64_t b = sdesc_sw128(smem_u32(sm.v[su][0]) + kk * 2048, 64 * 128, 1024);
-              mma_ts(tmem_o, tmem + su * 64 + kk * 8, b, IDESC_O, (u > 0 || kk > 0) ? 1u : 0u);
+              mma_ts_el(tmem_o, tmem + su * 64 + kk * 8, b, IDESC_O, (u > 0 || kk > 0) ? 1u : 0u);
             }
-            mma_commit(&sm.kv_empty[su]);
-            mma_commit(&sm.o_done);
+            mma_commit_el(&sm.kv_empty[su]);
+            mma_commit_el(&sm.o_done);
           }
         }
       }
       // drain: every MMA issued above completes before TMEM is released
-      mma_commit(&sm.drain);
+      mma_commit_el(&sm.drain);
       const WaitCtx drain_wc{&sm.never, nullptr, wait_limit_ns};
-      wait_bar(&sm.drain, 0, drain_wc);
+      wait_bar_all(&sm.drain, 0, drain_wc);
     }
   } else {
     // ---------------- softmax warps 0-3 ----------------

@@ -126,6 +126,18 @@ SPA2_DEV bool wait_bar(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
   }
 }
 
+// Waits for a warp that issues with the *_el calls: every lane waits (and so
+// takes the acquire itself); the result is true only when every lane saw the
+// phase, which keeps the caller's control flow warp-uniform.
+SPA2_DEV bool wait_bar_all(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
+  const bool ok = wait_bar(bar, parity, w);
+  return __all_sync(0xffffffffu, ok);
+}
+
+SPA2_DEV bool test_wait_all(uint64_t* bar, uint32_t parity) {
+  return __all_sync(0xffffffffu, mbar_test_wait(bar, parity));
+}
+
 // ---------------------------------------------------------------------------
 // TMA (tiled, no multicast)
 // ---------------------------------------------------------------------------
@@ -226,6 +238,43 @@ SPA2_DEV void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Warp-wide issue of tensor-core work. tcgen05.mma and tcgen05.commit act once
+// per executing thread. An issue loop run by a single lane keeps its operand
+// descriptors off the warp-uniform datapath and was measured to issue one
+// 128x64x16 product per ~70 cycles, where the tensor core finishes one in 48
+// (the 128 B/cycle it reads from shared memory); run by all 32 lanes, with
+// elect.sync choosing the lane that issues, the same loop keeps the tensor core
+// busy. Every lane must reach these calls together, so the caller keeps the
+// control flow around them warp-uniform (wait_bar_all / test_wait_all).
+SPA2_DEV void mma_ss_el(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+SPA2_DEV void mma_ts_el(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+SPA2_DEV void mma_commit_el(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
       : "memory");
 }
 
