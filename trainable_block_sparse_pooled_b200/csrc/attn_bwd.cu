@@ -680,7 +680,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_cons
 }
 
 // D = rowsum(dO * (O + O_lo)) in fp32; fp16 copies of the dO, V, Q and K rows
-// (|x| > 65504 clamped and reported). 16 threads per row.
+// (|x| > 65504 clamped and reported). D / 8 threads per row, 16-byte accesses.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
                                                       const __nv_bfloat16* __restrict__ o_lo,
@@ -691,49 +691,57 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __res
                                                       float* __restrict__ dvec, uint32_t* __restrict__ do16,
                                                       uint32_t* __restrict__ v16, uint32_t* __restrict__ q16,
                                                       uint32_t* __restrict__ k16, long long rows, int* status) {
-  constexpr int TPR = 16;
-  constexpr int EPT = D / TPR;  // 8 (d=128) or 4 (d=64) elements per thread
+  // one 16-byte access per tensor per thread (every tensor is 16-byte aligned
+  // and rows are D * 2 bytes): D / 8 threads per row, 8 elements each
+  constexpr int TPR = D / 8;
   const long long row = (long long)blockIdx.x * (256 / TPR) + threadIdx.x / TPR;
   const int tc = threadIdx.x % TPR;
   float acc = 0.f;
   bool bad = false;
   if (row < rows) {
-    const long long off = row * D + tc * EPT;
-#pragma unroll
-    for (int e = 0; e < EPT; e += 2) {
-      float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(o + off + e));
-      if (o_lo) {
-        const float2 l = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(o_lo + off + e));
-        a.x += l.x;
-        a.y += l.y;
-      }
-      float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(dout + off + e));
-      acc = fmaf(a.x, b.x, acc);
-      acc = fmaf(a.y, b.y, acc);
-      float2 w = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(v + off + e));
-      if (!(fabsf(b.x) <= 65504.f) || !(fabsf(b.y) <= 65504.f) || !(fabsf(w.x) <= 65504.f) ||
-          !(fabsf(w.y) <= 65504.f)) {
-        bad = true;
-        b.x = fminf(fmaxf(b.x, -65504.f), 65504.f);
-        b.y = fminf(fmaxf(b.y, -65504.f), 65504.f);
-        w.x = fminf(fmaxf(w.x, -65504.f), 65504.f);
-        w.y = fminf(fmaxf(w.y, -65504.f), 65504.f);
-      }
-      do16[(off + e) / 2] = pack_f16(b.x, b.y);
-      v16[(off + e) / 2] = pack_f16(w.x, w.y);
-      float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(q + off + e));
-      float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(k + off + e));
-      if (!(fabsf(x.x) <= 65504.f) || !(fabsf(x.y) <= 65504.f) || !(fabsf(y.x) <= 65504.f) ||
-          !(fabsf(y.y) <= 65504.f)) {
+    const long long off = row * D + tc * 8;
+    const uint4 ow = *reinterpret_cast<const uint4*>(o + off);
+    const uint4 lw = o_lo ? *reinterpret_cast<const uint4*>(o_lo + off) : make_uint4(0u, 0u, 0u, 0u);
+    const uint4 bw = *reinterpret_cast<const uint4*>(dout + off);
+    const uint4 vw = *reinterpret_cast<const uint4*>(v + off);
+    const uint4 qw = *reinterpret_cast<const uint4*>(q + off);
+    const uint4 kw = *reinterpret_cast<const uint4*>(k + off);
+    const uint32_t* O = reinterpret_cast<const uint32_t*>(&ow);
+    const uint32_t* L = reinterpret_cast<const uint32_t*>(&lw);
+    const uint32_t* Bd = reinterpret_cast<const uint32_t*>(&bw);
+    const uint32_t* Vv = reinterpret_cast<const uint32_t*>(&vw);
+    const uint32_t* Qq = reinterpret_cast<const uint32_t*>(&qw);
+    const uint32_t* Kk = reinterpret_cast<const uint32_t*>(&kw);
+    uint32_t d16[4], v16w[4], q16w[4], k16w[4];
+    auto f2 = [](uint32_t w) { return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w)); };
+    // fp16 copy of a bf16 pair; |x| > 65504 (or NaN) is clamped and flagged
+    auto to16 = [&bad](float2 x) {
+      if (!(fabsf(x.x) <= 65504.f) || !(fabsf(x.y) <= 65504.f)) {
         bad = true;
         x.x = fminf(fmaxf(x.x, -65504.f), 65504.f);
         x.y = fminf(fmaxf(x.y, -65504.f), 65504.f);
-        y.x = fminf(fmaxf(y.x, -65504.f), 65504.f);
-        y.y = fminf(fmaxf(y.y, -65504.f), 65504.f);
       }
-      q16[(off + e) / 2] = pack_f16(x.x, x.y);
-      k16[(off + e) / 2] = pack_f16(y.x, y.y);
+      return pack_f16(x.x, x.y);
+    };
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float2 a = f2(O[e]);
+      const float2 l = f2(L[e]);
+      a.x += l.x;
+      a.y += l.y;
+      const float2 b = f2(Bd[e]);
+      acc = fmaf(a.x, b.x, acc);
+      acc = fmaf(a.y, b.y, acc);
+      d16[e] = to16(b);
+      v16w[e] = to16(f2(Vv[e]));
+      q16w[e] = to16(f2(Qq[e]));
+      k16w[e] = to16(f2(Kk[e]));
     }
+    const long long w = off / 2;  // 32-bit word of the fp16 copies
+    *reinterpret_cast<uint4*>(do16 + w) = make_uint4(d16[0], d16[1], d16[2], d16[3]);
+    *reinterpret_cast<uint4*>(v16 + w) = make_uint4(v16w[0], v16w[1], v16w[2], v16w[3]);
+    *reinterpret_cast<uint4*>(q16 + w) = make_uint4(q16w[0], q16w[1], q16w[2], q16w[3]);
+    *reinterpret_cast<uint4*>(k16 + w) = make_uint4(k16w[0], k16w[1], k16w[2], k16w[3]);
   }
 #pragma unroll
   for (int s = TPR / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffff, acc, s);
@@ -745,7 +753,8 @@ template <int D>
 static cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
   const long long rows = (long long)a.BH * a.N;
   // 1. D and the fp16 copies of dO and V
-  bwd_pre_kernel<D><<<(unsigned)((rows + 15) / 16), 256, 0, s>>>(
+  constexpr int PRE_ROWS = 256 / (D / 8);  // rows per 256-thread block
+  bwd_pre_kernel<D><<<(unsigned)((rows + PRE_ROWS - 1) / PRE_ROWS), 256, 0, s>>>(
       (const __nv_bfloat16*)a.o, (const __nv_bfloat16*)a.o_lo, (const __nv_bfloat16*)a.dout,
       (const __nv_bfloat16*)a.v, (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, a.dvec, (uint32_t*)a.do16,
       (uint32_t*)a.v16, (uint32_t*)a.q16, (uint32_t*)a.k16, rows, a.status);
