@@ -127,6 +127,20 @@ static bool make_map(CUtensorMap* m, const void* ptr, const Shape& s, int rows, 
   return r == CUDA_SUCCESS;
 }
 
+// [BH, N, d] fp32 tensor, box {32, rows, 1} (128 bytes wide), 128-byte swizzle
+static bool make_map_f32(CUtensorMap* m, const void* ptr, const Shape& s, int rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)s.d, (cuuint64_t)s.N, (cuuint64_t)s.BH};
+  cuuint64_t strides[2] = {(cuuint64_t)s.d * 4, (cuuint64_t)s.N * s.d * 4};
+  cuuint32_t box[3] = {32, (cuuint32_t)rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 static int topk_count(float k_frac, int Tn) {
   long long K = (long long)floor((double)k_frac * (double)Tn + 0.5);
   if (K < 1) K = 1;
@@ -297,13 +311,13 @@ spa2_status spa2_sparse_attn_bwd(const void* q, const void* k, const void* v, co
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)d);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const bool f32 = grad_dtype == SPA2_DTYPE_F32;
-  CUtensorMap tq, tk, tv, tdo, tq16, tk16;
+  CUtensorMap tq, tk, tv, tdo, tq16, tk16, tdq;
   if (!make_map(&tq, q, s, 128) || !make_map(&tk, k, s, 64) || !make_map(&tv, w.v16, s, 64, true) ||
       !make_map(&tdo, w.do16, s, 128, true) || !make_map(&tq16, w.q16, s, 128, true) ||
-      !make_map(&tk16, w.k16, s, 64, true))
+      !make_map(&tk16, w.k16, s, 64, true) || !(f32 ? make_map_f32(&tdq, dq, s, 128) : make_map(&tdq, dq, s, 128)))
     return SPA2_ERR_CUDA;
   SPA2_CUDA_TRY(cudaMemsetAsync(w.status, 0, 4, st));
-  BwdArgs a{&tq, &tk, &tv, &tdo, &tq16, &tk16, q, k, o, o_lo, dout, v, lse, mask->row_cnt, mask->row_idx, mask->col_cnt,
+  BwdArgs a{&tq, &tk, &tv, &tdo, &tq16, &tk16, &tdq, q, k, o, o_lo, dout, v, lse, mask->row_cnt, mask->row_idx, mask->col_cnt,
             mask->col_idx, w.dvec, w.do16, w.v16, w.q16, w.k16, dq, dk, dv, f32 ? 1 : 0, (int)s.BH, s.N, s.Tm, s.Tn, scale,
             scale * 1.4426950408889634f, w.status, g_wait_limit_ns};
   SPA2_CUDA_TRY(launch_bwd(a, d, st));

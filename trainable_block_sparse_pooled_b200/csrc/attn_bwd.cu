@@ -437,12 +437,13 @@ struct DqSmem {
 template <int D>
 __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k,
                                                                const __grid_constant__ CUtensorMap tm_v16,
+                                                               const __grid_constant__ CUtensorMap tm_dq,
                                                                const __nv_bfloat16* __restrict__ qg,
                                                                const __half* __restrict__ do16,
                                                                const float* __restrict__ lse,
                                                                const float* __restrict__ dvec,
                                                                const int* __restrict__ row_cnt,
-                                                               const int* __restrict__ row_idx, void* __restrict__ dq,
+                                                               const int* __restrict__ row_idx,
                                                                int grad_f32, int N, int Tm, int Tn, float scale,
                                                                float scale_log2, int* status,
                                                                unsigned long long wait_limit_ns) {
@@ -496,6 +497,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_cons
     n = 0;
   }
   const int* kv_list = row_idx + rowid * Tn;
+  int epi_ok = 1;  // a dS thread clears it when its part of the dQ tile was not staged
 
   if (warp == 8) {
     // ---------------- TMA producer: the K / V ring ----------------
@@ -639,40 +641,55 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_cons
       tc_fence_before();
       mbar_arrive(&sm.ds_full[b]);
     }
-    // epilogue: dQ_i = scale * acc; warpgroup h writes feature columns h*D/2 .. +D/2
+    // epilogue: dQ_i = scale * acc, warpgroup h holding feature columns h*D/2 .. +D/2.
+    // The tile is staged in the K ring (idle once acc_done has fired: every product
+    // and every load is done) as 128-byte-swizzled boxes of 128 rows x 128 bytes
+    // (32 fp32 or 64 bf16 columns) and written by TMA stores below; the tensor
+    // map clips the rows of a ragged last q-block.
     if (ok) ok = wait_warp(&sm.acc_done, 0, wc);
     if (ok) {
       tc_fence_after();
+      uint8_t* stage = &sm.k[0][0][0];
 #pragma unroll 1
       for (int cc = 0; cc < D / 64; ++cc) {
-        const int c0 = h * (D / 2) + cc * 32;
+        const int c0 = h * (D / 2) + cc * 32;  // first feature column of this 32-column slice
         uint32_t a[32];
         tmem_ld32(tl + T_DQ + c0, a);
         tmem_wait_ld();
-        if (rvalid) {
-          const long long base = ((long long)bh * N + row) * D + c0;
-          if (grad_f32) {
-            float4* o = reinterpret_cast<float4*>(static_cast<float*>(dq) + base);
+        if (grad_f32) {
+          uint8_t* box = stage + (c0 / 32) * (128 * 128);
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              o[e] = make_float4(__uint_as_float(a[4 * e]) * scale, __uint_as_float(a[4 * e + 1]) * scale,
-                                 __uint_as_float(a[4 * e + 2]) * scale, __uint_as_float(a[4 * e + 3]) * scale);
-          } else {
-            uint4* o = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dq) + base);
+          for (int e = 0; e < 8; ++e)
+            *reinterpret_cast<float4*>(box + sw128_offset(r, e)) =
+                make_float4(__uint_as_float(a[4 * e]) * scale, __uint_as_float(a[4 * e + 1]) * scale,
+                            __uint_as_float(a[4 * e + 2]) * scale, __uint_as_float(a[4 * e + 3]) * scale);
+        } else {
+          uint8_t* box = stage + (c0 / 64) * (128 * 128);
+          const uint32_t u0 = (uint32_t)((c0 % 64) / 8);  // 16-byte unit of the slice in its 64-column box
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              o[e] = make_uint4(pack_bf16(__uint_as_float(a[8 * e]) * scale, __uint_as_float(a[8 * e + 1]) * scale),
-                                pack_bf16(__uint_as_float(a[8 * e + 2]) * scale, __uint_as_float(a[8 * e + 3]) * scale),
-                                pack_bf16(__uint_as_float(a[8 * e + 4]) * scale, __uint_as_float(a[8 * e + 5]) * scale),
-                                pack_bf16(__uint_as_float(a[8 * e + 6]) * scale, __uint_as_float(a[8 * e + 7]) * scale));
-          }
+          for (int e = 0; e < 4; ++e)
+            *reinterpret_cast<uint4*>(box + sw128_offset(r, u0 + e)) =
+                make_uint4(pack_bf16(__uint_as_float(a[8 * e]) * scale, __uint_as_float(a[8 * e + 1]) * scale),
+                           pack_bf16(__uint_as_float(a[8 * e + 2]) * scale, __uint_as_float(a[8 * e + 3]) * scale),
+                           pack_bf16(__uint_as_float(a[8 * e + 4]) * scale, __uint_as_float(a[8 * e + 5]) * scale),
+                           pack_bf16(__uint_as_float(a[8 * e + 6]) * scale, __uint_as_float(a[8 * e + 7]) * scale));
         }
       }
+      fence_proxy_async_smem();
     }
+    epi_ok = ok ? 1 : 0;
   }
 
   tc_fence_before();
-  __syncthreads();
+  // every thread takes part; the dQ tile is stored only when every dS thread staged its part
+  const int all_ok = __syncthreads_and(epi_ok);
+  if (threadIdx.x == 0 && all_ok && n > 0) {
+    const uint8_t* stage = &sm.k[0][0][0];
+    const int cols = grad_f32 ? 32 : 64;  // columns per 128-byte box
+    for (int b = 0; b < D / cols; ++b) tma_store_3d(&tm_dq, stage + b * (128 * 128), b * cols, i * 128, bh);
+    tma_store_commit();
+    tma_store_wait_all();
+  }
   if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -777,8 +794,8 @@ static cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
     e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     bwd_dq_kernel<D><<<dim3(a.Tm, a.BH), DQ_THREADS, smem, s>>>(
-        *a.tm_k, *a.tm_v, static_cast<const __nv_bfloat16*>(a.q), static_cast<const __half*>(a.do16), a.lse,
-        a.dvec, a.row_cnt, a.row_idx, a.dq, a.grad_f32, a.N, a.Tm, a.Tn, a.scale, a.scale_log2, a.status,
+        *a.tm_k, *a.tm_v, *a.tm_dq, static_cast<const __nv_bfloat16*>(a.q), static_cast<const __half*>(a.do16),
+        a.lse, a.dvec, a.row_cnt, a.row_idx, a.grad_f32, a.N, a.Tm, a.Tn, a.scale, a.scale_log2, a.status,
         a.wait_limit_ns);
     e = cudaGetLastError();
   }

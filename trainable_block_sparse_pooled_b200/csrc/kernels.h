@@ -51,6 +51,7 @@ struct BwdArgs {
   const CUtensorMap* tm_do;   // fp16 copy of dO, box {64, 128, 1}
   const CUtensorMap* tm_q16;  // fp16 copy of Q, box {64, 128, 1}
   const CUtensorMap* tm_k16;  // fp16 copy of K, box {64, 64, 1}
+  const CUtensorMap* tm_dq;   // dQ output: fp32 box {32, 128, 1} or bf16 box {64, 128, 1}, 128-byte swizzle
   const void* q;
   const void* k;
   const void* o;
