@@ -66,12 +66,14 @@ def test_ragged_fwd_bwd(N, d, kf, pf):
     _check_bwd(q, k, v, dense, dout, grads)
 
 
-def test_bf16_gradients_within_tolerance_plus_output_rounding():
+@pytest.mark.parametrize("d", [128, 64])
+def test_bf16_gradients_within_tolerance_plus_output_rounding(d):
     """bf16 gradient outputs: the stated tolerance plus half a bf16 ulp of each
-    expected value (the representation error of the output format itself)."""
-    q, k, v = synth.gaussian_with_sinks(B=1, H=2, N=1000, d=128, seed=12, device="cuda")
+    expected value (the representation error of the output format itself).
+    N = 1000 leaves a ragged last q-block (104 rows) and kv-block (40 rows)."""
+    q, k, v = synth.gaussian_with_sinks(B=1, H=2, N=1000, d=d, seed=12, device="cuda")
     dout = synth.normal_like(q.shape, seed=13, device="cuda")
-    s = b.Spa2(1, 2, 1000, 128)
+    s = b.Spa2(1, 2, 1000, d)
     m = s.block_mask(q, k, 0.1, 0.6)
     o, lse = s.fwd(q, k, v, m)
     g16 = s.bwd(q, k, v, o, lse, dout, m, grad_dtype=b.DTYPE_BF16)
