@@ -46,22 +46,34 @@ WORKLOADS = {
 }
 
 
+def code_digest(path):
+    """sha256 of a source file with its // comments and blank lines removed, so a
+    comment-only edit keeps a profile's counters attached to the same code."""
+    import hashlib
+    lines = []
+    with open(path, encoding="utf-8") as f:
+        for line in f:
+            code = line.split("//", 1)[0].rstrip()
+            if code:
+                lines.append(code)
+    return hashlib.sha256("\n".join(lines).encode()).hexdigest()
+
+
 def profiled_traffic(workload):
     """DRAM bytes (read + write) of one backward call on this workload, from the
     ncu summary under profiles/, or None when the summary is missing, covers
-    another workload, or was taken on a different backward source."""
-    import hashlib
+    another workload, or was taken on different backward code."""
     here = os.path.dirname(os.path.abspath(__file__))
     path = os.path.join(here, "profiles", "bwd_traffic.txt")
     src = os.path.join(here, "trainable_block_sparse_pooled_b200", "csrc", "attn_bwd.cu")
     try:
         fields = dict(line.split(":", 1) for line in open(path, encoding="utf-8")
                       if ":" in line and not line.startswith("#"))
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        digest = code_digest(src)
     except OSError:
         return None
     fields = {k.strip(): v.strip() for k, v in fields.items()}
-    if fields.get("source_sha256") != sha or fields.get("workload") != workload:
+    if fields.get("code_sha256") != digest or fields.get("workload") != workload:
         return None
     try:
         return int(fields["bytes_per_call"])

@@ -19,20 +19,27 @@
 //                  dS as fp16 tiles (11-bit significands; an fp16 dS keeps dK
 //                  within a few 1e-3 of the float64 result on the sink-key cases,
 //                  where a bf16 dS does not); warpgroup h handles kv columns
-//                  32h .. 32h+31, thread = query row. Warp 8: TMA producer; warp 9:
-//                  MMA issuer.
+//                  32h .. 32h+31, thread = query row. P / dS tiles are
+//                  double-buffered in shared memory, so tile t+1 is formed while
+//                  the tensor pipe runs dV/dK(t). Warp 8: TMA producer; warp 9:
+//                  MMA issuer, issuing whichever product is ready.
 // bwd_dq_kernel    one CTA per (q-block i, head), looping over the kv-blocks j
 //                  that i keeps (CSR row of i); recomputes S and dP, forms dS as a
 //                  hi + lo pair of bf16 values (about 16 significant bits: dQ is
 //                  the gradient most sensitive to dS rounding) and accumulates
 //                  dQ_i = sum_j dS_ij K_j in TMEM
 //                    dQ  += dS K_j      bf16  M=128 (q) N=d       K=64   A K-, B MN-major
-//                  then writes it once: no atomics and no fp32 scratch for dQ.
+//                  then writes it once (staged in shared memory, TMA stores): no
+//                  atomics and no fp32 scratch for dQ.
 //                  For d = 64 the dV^T / dK^T MMAs still run at M = 128 (the
 //                  upper 64 lanes repeat the lower ones and are ignored).
 //
 // TMEM columns (both kernels): S[2] 0..127, dP[2] 128..255; dV^T 256..319 and
 // dK^T 320..383 (dkdv), dQ 256..256+d (dq).
+// In both kernels the MMA warp runs its issue loop with all 32 lanes and
+// elect.sync picks the lane that issues each tcgen05.mma / tcgen05.commit (the
+// descriptor arithmetic then stays on the warp-uniform datapath; a one-lane loop
+// could not keep up with the tensor core).
 #include <algorithm>
 
 #include "common.cuh"

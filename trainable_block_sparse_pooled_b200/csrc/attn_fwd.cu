@@ -6,14 +6,16 @@
 // kv-blocks j (b_kv = 64 rows each) listed in the CSR row of i.
 //
 //   warp 4      TMA producer: Q_i once, then K_j / V_j through a 2-slot ring.
-//   warp 5      MMA issuer (one thread): S = Q K_j^T (SS, bf16, M=128 N=64 K=d)
+//   warp 5      MMA issuer (all 32 lanes run the loop, elect.sync picks the lane
+//               that issues each tcgen05 op): S = Q K_j^T (SS, bf16, M=128 N=64 K=d)
 //               into one of two TMEM S buffers; O += P V_j (TS: P from TMEM,
 //               fp16 operands, M=128 N=d K=64). Owns the 256-column TMEM
 //               allocation.
 //   warps 0-3   softmax, thread t <-> query row t <-> TMEM lane t: load S,
 //               online max / exp2 / sum in registers, write P (fp16, values in
-//               [0, 256]: 8x finer rounding than bf16) over the S buffer, rescale O in TMEM only when the running max grew by
-//               more than 2^8 (lazy rescale), then the epilogue O / l -> bf16
+//               [0, 256]: 8x finer rounding than bf16) over the S buffer,
+//               rescale O in TMEM only when the running max grew by more than
+//               2^8 (lazy rescale), then the epilogue O / l -> bf16
 //               (and optionally its bf16 residual) -> smem -> TMA store, LSE.
 //
 // TMEM columns: [0,64) S/P buffer 0, [64,128) S/P buffer 1, [128,128+d) O.
