@@ -87,3 +87,44 @@ def test_row_type_ordering_on_mixed_rows(target):
     assert tk["skewed"] < tp["skewed"]          # sink rows: the threshold is met too early
     assert hy["uniform"] < tk["uniform"]        # the hybrid avoids both failures
     assert hy["skewed"] < tp["skewed"]
+
+
+class _OracleSpa2:
+    """CPU stand-in for binding.Spa2 with the oracle behind block_mask / fwd, so
+    that ablation.row_type_errors' own logic (strategy parameters, row labels,
+    means) runs without a GPU. Test infrastructure only."""
+
+    class _Mask:
+        def __init__(self, dense):
+            self.dense = dense
+
+        def kept_blocks(self):
+            return int(self.dense.sum())
+
+    def __init__(self, Q, K, V):
+        self.torch = torch
+        self.Q, self.K, self.V = Q, K, V
+        self.B, self.H, self.N, self.d = Q.shape
+        self.Tm, self.Tn = O.block_counts(self.N, BQ, BKV)
+
+    def block_mask(self, q, k, k_frac, p_frac):
+        return self._Mask(O.block_mask(self.Q, self.K, BQ, BKV, k_frac, p_frac)[2])
+
+    def fwd(self, q, k, v, mask, want_o_lo=True):
+        _, lse = O.masked_attn_fwd(self.Q, self.K, self.V, mask.dense, BQ, BKV)
+        return None, torch.from_numpy(lse)
+
+    def check(self):
+        pass
+
+
+def test_row_type_errors_aggregation_matches_direct_computation():
+    q, k, v = synth.mixed_rows(B=1, H=1, N=4096, d=128, seed=4, grid=(4, 32, 32))
+    Q, K, V = _f64(q), _f64(k), _f64(v)
+    spa = _OracleSpa2(Q, K, V)
+    got = ablation.row_type_errors(spa, torch.zeros(0), torch.zeros(0), torch.zeros(0), 0.9)
+    want = _oracle_errors(Q, K, V, 0.9)
+    for st in ablation.STRATEGIES:
+        assert got[st]["sparsity"] == pytest.approx(want[st]["sparsity"], abs=1e-12)
+        for lab in ("uniform", "skewed"):
+            assert got[st][lab] == pytest.approx(want[st][lab], abs=1e-9), (st, lab)
