@@ -21,7 +21,7 @@ Attention via Hybrid Top-k+Top-p Masking and Distillation Fine-Tuning"):
 * [chatpaper] chatpaper.ai abstract ("efficient trainable sparse attention
   implementation": forward and backward).
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 
 * pool = arithmetic mean over the rows of a block; the last block of a ragged
   sequence is averaged over its valid rows only.

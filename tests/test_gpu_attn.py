@@ -127,7 +127,7 @@ def test_forward_is_deterministic():
 
 
 def test_mixed_rows_fwd_bwd_small():
-    """Config-3 recipe (near-uniform even q-blocks, +6-logit skewed odd q-blocks,
+    """Mixed-rows recipe (near-uniform even q-blocks, +6-logit skewed odd q-blocks,
     k=5% p=90%) on the 8x32x32 grid, whole heads, forward and backward."""
     q, k, v = synth.mixed_rows(B=1, H=2, N=8192, d=128, seed=4, device="cuda", grid=(8, 32, 32))
     dout = synth.normal_like(q.shape, seed=5, device="cuda")
@@ -163,7 +163,7 @@ def test_wan13b_fwd_sampled_qblocks():
 
 @pytest.mark.slow
 def test_wan13b_bwd_sampled_blocks():
-    """1.3B shape, mixed rows (config-3 recipe), k=5% p=90%, forward + backward:
+    """1.3B shape, mixed rows, k=5% p=90%, forward + backward:
     dQ of 8 sampled q-blocks and dK, dV of 8 sampled kv-blocks (the last, ragged,
     one included) in heads 0 and 11, against the oracle."""
     q, k, v = synth.mixed_rows(B=1, H=12, N=32760, d=128, seed=2, device="cuda")

@@ -5,7 +5,7 @@ arithmetic, and both the CUDA path and the float64 oracle consume what it
 returns. Everything is generated with torch from explicit seeds, then rounded
 to bf16 (round-to-nearest-even) so both sides see identical bits.
 
-Generators (the recipes are stated in DESIGN.md, "Inputs"):
+Generators:
 
 * ``gaussian_with_sinks``  N(0, 1) Q/K/V plus key "sink" tokens whose norm is 8x
   the mean key norm, pointing along the head's mean query (small parity case).
