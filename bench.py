@@ -230,13 +230,15 @@ def run_reference(args, wl, name):
     import oracle
     from trainable_block_sparse_pooled_b200 import calibrate
     torch.set_num_threads(os.cpu_count() or 1)
-    q, k, v, dout = make_inputs(dict(wl, H=1), seed=0, device="cpu")   # head 0 of the layer
-    # calibrate p on head 0 with the oracle's own mask (the GPU arm calibrates all heads)
-    Qb = oracle.pool_blocks(q.float().numpy().astype(np.float64), 128)
-    Kb = oracle.pool_blocks(k.float().numpy().astype(np.float64), 64)
+    qa, ka, va, da = make_inputs(wl, seed=0, device="cpu")               # every head of the layer
+    # calibrate p over all heads with the oracle's own mask, as the GPU arm does with its kernels
+    Qb = oracle.pool_blocks(qa.float().numpy().astype(np.float64), 128)
+    Kb = oracle.pool_blocks(ka.float().numpy().astype(np.float64), 64)
     pbar32 = oracle.pooled_attention(Qb, Kb, wl["d"]).astype(np.float32)
     kf, pf, _ = calibrate.calibrate_p(lambda a, c: int(oracle.select_blocks(pbar32, a, c).sum()), pbar32.size,
-                                      args.target_sparsity, tol=0.01, iters=12)
+                                      args.target_sparsity)
+    q, k, v, dout = (x[:, :1].contiguous() for x in (qa, ka, va, da))   # head 0 is the timed sample
+    del qa, ka, va, da
     per_step_s = 4.0
     for _ in range(args.warmup):
         cpu_oracle_sample(q, k, v, dout, kf, pf, per_step_s / 4, max_blocks=2)
