@@ -11,7 +11,7 @@ import oracle
 from tests._parity import assert_close, assert_close_bf16_out, csr_to_dense, f64
 from trainable_block_sparse_pooled_b200 import binding as b
 from trainable_block_sparse_pooled_b200 import synth
-from trainable_block_sparse_pooled_b200.autograd import sparse_attention
+from trainable_block_sparse_pooled_b200.autograd import block_mask, sparse_attention
 
 pytestmark = pytest.mark.gpu
 
@@ -34,6 +34,32 @@ def test_autograd_gradients_match_oracle():
     for name, g, e in (("dQ", qg.grad, dQ), ("dK", kg.grad, dK), ("dV", vg.grad, dV)):
         assert g.dtype == torch.bfloat16
         assert_close_bf16_out(f64(g), e, name)
+
+
+def test_reused_mask():
+    """A mask built once with block_mask and passed to later calls: on the same
+    inputs it reproduces the call that builds its own mask bit for bit (both
+    passes are deterministic); on another step's inputs it matches the oracle
+    under that same mask."""
+    q, k, v = synth.gaussian_with_sinks(B=1, H=2, N=1000, d=128, seed=31, device="cuda")
+    dout = synth.normal_like(q.shape, seed=32, device="cuda")
+    m = block_mask(q, k, 0.2, 0.6)
+    runs = []
+    for kw in (dict(k_frac=0.2, p_frac=0.6), dict(mask=m)):
+        qg, kg, vg = (t.clone().requires_grad_(True) for t in (q, k, v))
+        o = sparse_attention(qg, kg, vg, **kw)
+        (o.float() * dout.float()).sum().backward()
+        runs.append((o.detach(), qg.grad, kg.grad, vg.grad))
+    for a, c in zip(*runs):
+        assert torch.equal(a, c)
+    # another diffusion step: new q, k, v of the same shape, the mask of the first
+    q2, k2, v2 = synth.gaussian_with_sinks(B=1, H=2, N=1000, d=128, seed=33, device="cuda")
+    o2 = sparse_attention(q2, k2, v2, mask=m)
+    dense = csr_to_dense(m.row_cnt.cpu().numpy(), m.row_idx.cpu().numpy(), m.row_idx.shape[-1])
+    O2, _ = oracle.masked_attn_fwd(f64(q2), f64(k2), f64(v2), dense, 128, 64)
+    assert_close_bf16_out(f64(o2), O2, "O (bf16), reused mask")
+    with pytest.raises(ValueError):
+        sparse_attention(q2[:, :1].contiguous(), k2[:, :1].contiguous(), v2[:, :1].contiguous(), mask=m)
 
 
 class _AttnBlock(torch.nn.Module):

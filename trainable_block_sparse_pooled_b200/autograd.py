@@ -7,6 +7,10 @@ through the same mask, which the method holds constant (its trainable part is
 the attention itself: chatpaper.ai abstract (ii)). Every step runs in the
 libspa2 kernels; this module only marshals arguments through the C ABI
 (`binding.Spa2`) and caches the per-shape workspaces.
+
+A mask can also be built once with `block_mask(q, k, k_frac, p_frac)` and
+passed as `sparse_attention(..., mask=m)` to later calls of the same shape
+(other diffusion steps or layers), which then skip pooling and selection.
 """
 
 from __future__ import annotations
@@ -35,18 +39,23 @@ class SparseAttentionFunction(torch.autograd.Function):
     """
 
     @staticmethod
-    def forward(ctx, q, k, v, k_frac: float, p_frac: float, scale: float = 0.0):
+    def forward(ctx, q, k, v, k_frac: float, p_frac: float, scale: float = 0.0, mask: b.Mask | None = None):
         if q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16 or v.dtype != torch.bfloat16:
             raise TypeError("sparse_attention expects bf16 q, k, v")
         q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
         B, H, N, d = q.shape
         s = _spa(B, H, N, d, q.device)
-        mask = s.block_mask(q, k, k_frac, p_frac)
+        if mask is None:
+            mask = s.block_mask(q, k, k_frac, p_frac)
+        elif tuple(mask.row_cnt.shape) != (B, H, s.Tm) or tuple(mask.row_idx.shape) != (B, H, s.Tm, s.Tn) \
+                or mask.col_cnt is None or mask.row_cnt.device != q.device:
+            raise ValueError("mask does not belong to a problem of this shape and device")
         o, lse = s.fwd(q, k, v, mask, scale)
         ctx.save_for_backward(q, k, v, o, lse, s.o_lo)
         ctx.mask, ctx.scale, ctx.spa = mask, scale, s
-        ctx.mark_non_differentiable(mask.row_cnt)
-        return o, mask.row_cnt  # the kept-block counts, so callers can see the mask
+        row_cnt = mask.row_cnt.clone()  # the kept-block counts (a copy: a reused mask serves many calls)
+        ctx.mark_non_differentiable(row_cnt)
+        return o, row_cnt
 
     @staticmethod
     def backward(ctx, do, _row_cnt_grad):
@@ -54,10 +63,25 @@ class SparseAttentionFunction(torch.autograd.Function):
         dq, dk, dv = ctx.spa.bwd(q, k, v, o, lse, do.contiguous(), ctx.mask, ctx.scale, o_lo=o_lo,
                                  grad_dtype=b.DTYPE_BF16)
         ctx.spa.check()  # device-side errors of the mask, forward and backward of this call
-        return dq, dk, dv, None, None, None
+        return dq, dk, dv, None, None, None, None
 
 
-def sparse_attention(q, k, v, k_frac: float, p_frac: float, scale: float = 0.0, return_mask: bool = False):
-    """Differentiable hybrid block-sparse attention (b_q = 128, b_kv = 64)."""
-    o, row_cnt = SparseAttentionFunction.apply(q, k, v, k_frac, p_frac, scale)
+def block_mask(q, k, k_frac: float, p_frac: float) -> b.Mask:
+    """The hybrid block mask of (q, k) alone (CSR and CSC on the device), for
+    reuse through `sparse_attention(..., mask=...)`."""
+    if q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16:
+        raise TypeError("block_mask expects bf16 q, k")
+    q, k = q.contiguous(), k.contiguous()
+    B, H, N, d = q.shape
+    return _spa(B, H, N, d, q.device).block_mask(q, k, k_frac, p_frac)
+
+
+def sparse_attention(q, k, v, k_frac: float = 0.0, p_frac: float = 0.0, scale: float = 0.0,
+                     return_mask: bool = False, mask: b.Mask | None = None):
+    """Differentiable hybrid block-sparse attention (b_q = 128, b_kv = 64).
+
+    With `mask` (from `block_mask` on a problem of the same shape) the given
+    mask is used as is and k_frac, p_frac are ignored.
+    """
+    o, row_cnt = SparseAttentionFunction.apply(q, k, v, k_frac, p_frac, scale, mask)
     return (o, row_cnt) if return_mask else o
