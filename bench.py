@@ -46,17 +46,17 @@ WORKLOADS = {
 }
 
 
-def code_digest(path):
-    """sha256 of a source file with its // comments and blank lines removed, so a
+def code_text_digest(text):
+    """sha256 of source text with its // comments and blank lines removed, so a
     comment-only edit keeps a profile's counters attached to the same code."""
     import hashlib
-    lines = []
+    lines = [ln.split("//", 1)[0].rstrip() for ln in text.splitlines()]
+    return hashlib.sha256("\n".join(ln for ln in lines if ln).encode()).hexdigest()
+
+
+def code_digest(path):
     with open(path, encoding="utf-8") as f:
-        for line in f:
-            code = line.split("//", 1)[0].rstrip()
-            if code:
-                lines.append(code)
-    return hashlib.sha256("\n".join(lines).encode()).hexdigest()
+        return code_text_digest(f.read())
 
 
 def profiled_traffic(workload):

@@ -26,3 +26,13 @@ def test_calibration_hits_target_with_oracle_counts():
 def test_calibration_returns_topk_only_when_target_is_loose():
     kf, pf, s = calibrate.calibrate_p(lambda k, p: 10, 100, 0.95)
     assert pf == 0.0 and abs(s - 0.9) < 1e-12
+
+
+def test_code_digest_ignores_comments_but_not_code():
+    import bench
+    src = "int f(int x) {\n  return x + 1;  // add one\n}\n"
+    same = "// header\nint f(int x) {\n\n  return x + 1;  // plus one\n}\n"
+    changed = "int f(int x) {\n  return x + 2;  // add one\n}\n"
+    assert bench.code_text_digest(src) == bench.code_text_digest(same)
+    assert bench.code_text_digest(src) != bench.code_text_digest(changed)
+
