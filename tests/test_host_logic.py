@@ -36,3 +36,28 @@ def test_code_digest_ignores_comments_but_not_code():
     assert bench.code_text_digest(src) == bench.code_text_digest(same)
     assert bench.code_text_digest(src) != bench.code_text_digest(changed)
 
+
+
+def test_calibration_bisection_property():
+    """For any kept-count curve that grows continuously in p (here a + (1 - a) p^g
+    of a million blocks), the bisection lands within its tolerance of every
+    target that Top-k alone overshoots."""
+    from hypothesis import given, settings, strategies as st
+
+    @settings(max_examples=200, deadline=None)
+    @given(a=st.floats(0.001, 0.5), g=st.floats(0.2, 5.0), target=st.floats(0.05, 0.95))
+    def check(a, g, target):
+        total = 1_000_000
+
+        def kept(k, p):
+            return int(total * (a + (1.0 - a) * p ** g))
+
+        kf, pf, s = calibrate.calibrate_p(kept, total, target)
+        assert 0.0 <= pf <= 1.0
+        assert s == 1.0 - kept(kf, pf) / total
+        if 1.0 - a > target + 0.0025:
+            assert abs(s - target) <= 0.0025
+        else:
+            assert pf == 0.0
+
+    check()
