@@ -59,13 +59,23 @@ def code_digest(path):
         return code_text_digest(f.read())
 
 
-def profiled_traffic(workload):
-    """DRAM bytes (read + write) of one backward call on this workload, from the
-    ncu summary under profiles/, or None when the summary is missing, covers
-    another workload, or was taken on different backward code."""
-    here = os.path.dirname(os.path.abspath(__file__))
-    path = os.path.join(here, "profiles", "bwd_traffic.txt")
-    src = os.path.join(here, "trainable_block_sparse_pooled_b200", "csrc", "attn_bwd.cu")
+KERNEL_SOURCES = {
+    "pool_kernel": "mask.cu", "select_kernel": "mask.cu", "csc_kernel": "mask.cu",
+    "v_to_f16_kernel": "attn_fwd.cu", "fwd_kernel": "attn_fwd.cu",
+    "bwd_pre_kernel": "attn_bwd.cu", "bwd_dkdv_kernel": "attn_bwd.cu", "bwd_dq_kernel": "attn_bwd.cu",
+}
+
+
+def profiled_traffic(kernel, workload):
+    """DRAM bytes (read + write) per launch of `kernel` on this workload, from the
+    ncu summary profiles/traffic_<kernel>.txt, or None when the summary is missing,
+    covers another workload, or was taken on different code (the digest of the
+    kernel's source file, comments and blank lines removed, must match)."""
+    src_name = KERNEL_SOURCES.get(kernel)
+    if src_name is None:
+        return None
+    path = os.path.join(ROOT, "profiles", f"traffic_{kernel}.txt")
+    src = os.path.join(ROOT, "trainable_block_sparse_pooled_b200", "csrc", src_name)
     try:
         fields = dict(line.split(":", 1) for line in open(path, encoding="utf-8")
                       if ":" in line and not line.startswith("#"))
@@ -76,9 +86,50 @@ def profiled_traffic(workload):
     if fields.get("code_sha256") != digest or fields.get("workload") != workload:
         return None
     try:
-        return int(fields["bytes_per_call"])
+        return int(fields["bytes_per_launch"])
     except (KeyError, ValueError):
         return None
+
+
+def clock_scaled_peak(pk, clk):
+    """bf16 tensor peak for a kernel timed at this run's clocks: the burst peak
+    (taken at the maximum SM clock) scaled by median / maximum SM clock of the
+    samples taken during the timed region, never above the burst peak."""
+    burst = pk["bf16_tflops"]
+    med, top = clk.get("sm_mhz"), clk.get("sm_max_mhz") or pk.get("sm_max_mhz")
+    if not med or not top:
+        return burst, "burst (no clock samples)"
+    ratio = min(1.0, med / top)
+    if ratio >= 0.99:
+        return burst, f"burst: SM clock median {med:.0f} of {top:.0f} MHz"
+    return burst * ratio, f"burst x {ratio:.3f} (SM clock median {med:.0f} of {top:.0f} MHz)"
+
+
+def kernel_work(name, B, H, N, d, Tm, Tn, kept, fwd_flops):
+    """Algorithmic work of one launch of a library kernel on this layer:
+    (bound, amount, unit) with unit 'flop' for tensor-core kernels (forward
+    4 d per kept token pair; the dK/dV pass holds 4 of the backward's 5
+    products, the dQ pass 1) and 'byte' for HBM-bound kernels (every input read
+    once, every output written once)."""
+    e = B * H * N * d
+    if name == "fwd_kernel":
+        return "tensor", fwd_flops, "flop"
+    if name == "bwd_dkdv_kernel":
+        return "tensor", 2.0 * fwd_flops, "flop"
+    if name == "bwd_dq_kernel":
+        return "tensor", 0.5 * fwd_flops, "flop"
+    if name == "pool_kernel":
+        return "hbm", 2.0 * e * 2 + 4.0 * B * H * (Tm + Tn) * d, "byte"
+    if name == "select_kernel":
+        return "hbm", 4.0 * B * H * (Tm + Tn) * d + 4.0 * (kept + B * H * Tm) + 4.0 * B * H * Tm * ((Tn + 31) // 32), \
+            "byte"
+    if name == "csc_kernel":
+        return "hbm", 4.0 * B * H * Tm * ((Tn + 31) // 32) + 4.0 * (kept + B * H * Tn), "byte"
+    if name == "v_to_f16_kernel":
+        return "hbm", 4.0 * e, "byte"
+    if name == "bwd_pre_kernel":
+        return "hbm", 20.0 * e + 4.0 * B * H * N, "byte"
+    return None, 0.0, None
 
 
 def peaks():
@@ -178,13 +229,14 @@ def make_inputs(wl, seed, device):
     return q.contiguous(), k.contiguous(), v.contiguous(), dout.contiguous()
 
 
-def kept_flops(mask, N, d):
-    """Forward flops 4*d*sum over kept (i, j) of valid rows x valid cols (torch, on device)."""
+def kept_flops(mask, N, d, bq=128, bkv=64):
+    """Forward flops 4*d*sum over kept (i, j) of valid rows x valid cols, from the
+    CSR form of the mask (torch, on the mask's device)."""
     import torch
     dev = mask.row_cnt.device
     Tm, Tn = mask.row_idx.shape[-2], mask.row_idx.shape[-1]
-    rows = (torch.clamp(N - torch.arange(Tm, device=dev) * 128, max=128)).double()
-    cols = (torch.clamp(N - torch.arange(Tn, device=dev) * 64, max=64)).double()
+    rows = (torch.clamp(N - torch.arange(Tm, device=dev) * bq, max=bq)).double()
+    cols = (torch.clamp(N - torch.arange(Tn, device=dev) * bkv, max=bkv)).double()
     valid = torch.arange(Tn, device=dev) < mask.row_cnt[..., None]
     idx = mask.row_idx.long().clamp(0, Tn - 1)
     colsum = (cols[idx] * valid).sum(-1)
@@ -338,7 +390,6 @@ def run_gpu(args, wl, name):
     dq = torch.empty(q.shape, dtype=gt, device=dev)
     dk = torch.empty(q.shape, dtype=gt, device=dev)
     dv = torch.empty(q.shape, dtype=gt, device=dev)
-    launches_per_step = 3 + 2 + 3   # pool, select, csc | V->fp16, fwd | D + fp16 copies, dK/dV, dQ
 
     def step(ev=None):
         if ev is not None:
@@ -369,12 +420,16 @@ def run_gpu(args, wl, name):
     clocks.start()
     time.sleep(0.15)
     torch.cuda.nvtx.range_push("spa2_timed")     # ncu --nvtx-include "spa2_timed/" selects this region
+    b.spa2_timing_read()                         # forget launches recorded before the timed region
+    b.spa2_timing_enable(True)                   # per-kernel CUDA events on the launch stream
     t_start.record()
     for i in range(args.steps):
         step(evs[i])
     t_end.record()
     torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
+    b.spa2_timing_enable(False)
+    per_kernel = b.spa2_timing_read()
     clk = clocks.stop()
     barrier(dist)
     s.check()
@@ -440,8 +495,24 @@ def run_gpu(args, wl, name):
     value = step_flops * ws / (ms * 1e-3) / 1e12
     bwd_tf = bwd_flops / (bwd_ms * 1e-3) / 1e12
     fwd_tf = fwd_flops / (fwd_ms * 1e-3) / 1e12
-    mask_bytes = 2.0 * B * H * N * d * 2 + 4.0 * (B * H * s.Tm + int(mask.row_cnt.sum().item()) * 2 + B * H * s.Tn)
+    kept = int(mask.row_cnt.sum().item())
+    mask_bytes = 2.0 * B * H * N * d * 2 + 4.0 * (B * H * s.Tm + kept * 2 + B * H * s.Tn)
     mask_gbs = mask_bytes / (mask_ms * 1e-3) / 1e9
+    tensor_peak, tensor_peak_kind = clock_scaled_peak(pk, clk)
+    kernels = {}
+    for kname, (n_launch, tot_ms) in per_kernel.items():
+        bound, work, unit = kernel_work(kname, B, H, N, d, s.Tm, s.Tn, kept, fwd_flops)
+        avg_ms = tot_ms / n_launch
+        ent = {"launches": n_launch, "avg_us": avg_ms * 1e3, "share": tot_ms / (ms * args.steps)}
+        if bound == "tensor":
+            ent.update(bound="tensor", achieved=work / (avg_ms * 1e-3) / 1e12, unit="TFLOP/s")
+            ent["frac"] = ent["achieved"] / tensor_peak
+        elif bound == "hbm":
+            ent.update(bound="hbm", achieved=work / (avg_ms * 1e-3) / 1e9, unit="GB/s")
+            ent["frac"] = ent["achieved"] / pk["hbm_gbs"]
+        kernels[kname] = ent
+    dom = max(kernels, key=lambda k: kernels[k]["share"])
+    dk = kernels[dom]
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -453,18 +524,24 @@ def run_gpu(args, wl, name):
                              "seeded N(0,1) with 2 sink keys, dO ~ N(0,1)",
                    "grad_dtype": "fp32", "l2": "inputs larger than L2 (Q, K, V, dO are 4 x %.0f MB)" %
                    (B * H * N * d * 2 / 1e6), "parallelism": f"independent layer per GPU x{ws}"},
-        "roofline": {"bound": "tensor", "kernel": "backward call: D pre-pass + bwd_dkdv_kernel + bwd_dq_kernel",
-                     "achieved": bwd_tf, "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                     "frac": bwd_tf / pk["bf16_tflops_sustained"], "traffic": profiled_traffic(name),
-                     "peak_kind": f"{pk_kind} bf16 sustained (kernel timed inside a long step)"},
+        "roofline": {"bound": dk.get("bound"), "kernel": dom, "achieved": dk.get("achieved"),
+                     "peak": tensor_peak if dk.get("bound") == "tensor" else pk["hbm_gbs"],
+                     "unit": dk.get("unit"), "frac": dk.get("frac"),
+                     "traffic": profiled_traffic(dom, name),
+                     "avg_launch_us": dk["avg_us"], "share_of_step": dk["share"],
+                     "peak_kind": (f"{pk_kind} bf16 {tensor_peak_kind}" if dk.get("bound") == "tensor"
+                                   else f"{pk_kind} HBM copy bandwidth")},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": sum(v["launches"] for v in kernels.values()),
         "clocks": clk,
+        "kernels": kernels,
         "ops": {"mask_us": mask_ms * 1e3, "mask_GBps": mask_gbs, "mask_hbm_frac": mask_gbs / pk["hbm_gbs"],
-                "fwd_ms": fwd_ms, "fwd_tflops": fwd_tf, "fwd_frac_burst": fwd_tf / pk["bf16_tflops"],
-                "bwd_ms": bwd_ms, "bwd_tflops": bwd_tf, "bwd_frac_burst": bwd_tf / pk["bf16_tflops"],
-                "fwd_flops": fwd_flops, "bwd_flops": bwd_flops},
+                "fwd_ms": fwd_ms, "fwd_tflops": fwd_tf, "fwd_frac": fwd_tf / tensor_peak,
+                "bwd_ms": bwd_ms, "bwd_tflops": bwd_tf, "bwd_frac": bwd_tf / tensor_peak,
+                "fwd_flops": fwd_flops, "bwd_flops": bwd_flops,
+                "note": "per-op times are CUDA events around each C-ABI call in the timed steps; fractions "
+                        "use the clock-scaled burst peak of roofline.peak_kind"},
         "dense": dense,
     }
     if rank == 0:

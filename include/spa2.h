@@ -143,10 +143,15 @@ SPA2_API spa2_status spa2_block_mask(const void* q, const void* k, int B, int H,
  *            refused with SPA2_ERR_WORKSPACE before any launch.
  *   setup:   the first call on a device (with that device current) looks the
  *            array's address up once and caches it; make that first call
- *            before any stream capture begins on that device.
+ *            before any stream capture begins on that device. A
+ *            cudaDeviceReset unloads the library's device image, and with it
+ *            the array: calls on that device after a reset are not supported
+ *            (the cached address is stale).
  *   status:  NULL, or a 4-byte-aligned device int the caller owns; the call
  *            copies the device-side status word there (stream-ordered). Read
- *            it with spa2_stream_status(status, stream).
+ *            it with spa2_stream_status(status, stream). With status == NULL
+ *            device-side errors of the call (a timed-out wait, a failed bounds
+ *            check) are discarded: nothing reports them.
  *   races:   all calls on one device share the array. Calls issued one after
  *            another on one stream are safe; calls whose executions overlap
  *            (other streams, other host threads) race and give wrong masks.
@@ -248,6 +253,29 @@ SPA2_API spa2_status spa2_debug_set_wait_limit_ns(long long limit);
  * bytes) and returns normally, leaving the context usable.
  */
 SPA2_API spa2_status spa2_debug_timeout_probe(void* ws, size_t ws_bytes, spa2_stream_t stream);
+
+/*
+ * Per-kernel timing, a measurement aid with no counterpart in the method.
+ * While timing is on, every kernel the library launches is bracketed by two
+ * CUDA events recorded on its launch stream (this adds a few microseconds of
+ * event records per call and nothing else; results are unchanged). Events are
+ * created on demand (cudaEventCreate; no device memory) and recycled.
+ *   spa2_timing_enable(on)  on != 0 starts recording, 0 stops; returns SPA2_OK.
+ *   spa2_kernel_count()     number of kernel kinds (ids 0 .. count-1).
+ *   spa2_kernel_name(id)    static name of kernel kind `id` ("unknown" if out of range).
+ *   spa2_timing_read(n, launches, total_ms)
+ *                           waits for every event recorded since the last read,
+ *                           writes for ids 0 .. n-1 the number of launches and
+ *                           their summed event time in milliseconds (host arrays
+ *                           of n entries), then forgets the recorded launches.
+ *                           SPA2_ERR_CUDA if an event could not be read (e.g.
+ *                           it was recorded during stream capture);
+ *                           SPA2_ERR_INVALID_ARG for n < 0 or NULL arrays.
+ */
+SPA2_API spa2_status spa2_timing_enable(int on);
+SPA2_API int spa2_kernel_count(void);
+SPA2_API const char* spa2_kernel_name(int kernel_id);
+SPA2_API spa2_status spa2_timing_read(int n, int* launches, double* total_ms);
 
 #ifdef __cplusplus
 }

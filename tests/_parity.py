@@ -62,6 +62,28 @@ class Accum:
         return self.ma, rl1
 
 
+class AccumBf16(Accum):
+    """Accum for a bf16 output: per element |err| <= max_abs + half a bf16 ulp of
+    the expected value (the output format's own rounding), and the same
+    relative-L1 bound as every other output, summed over all sampled blocks."""
+
+    def __init__(self, what):
+        super().__init__(what)
+        self.excess = -np.inf
+
+    def add(self, actual, expected):
+        super().add(actual, expected)
+        e = np.asarray(expected, dtype=np.float64)
+        d = np.abs(np.asarray(actual, dtype=np.float64) - e)
+        self.excess = max(self.excess, float((d - bf16_half_ulp(e)).max()))
+
+    def check(self, max_abs=MAX_ABS, rel_l1=REL_L1):
+        rl1 = self.err / max(self.ref, 1e-300)
+        assert self.excess <= max_abs and rl1 <= rel_l1, \
+            f"{self.what}: max excess over half an ulp={self.excess:.3e} rel_l1={rl1:.3e}"
+        return self.excess, rl1
+
+
 def csr_to_dense(row_cnt, row_idx, Tn):
     """bool [.., Tm, Tn] from CSR numpy arrays; checks ids ascending and in range."""
     cnt = np.asarray(row_cnt)

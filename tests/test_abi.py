@@ -97,3 +97,14 @@ def test_argument_errors_are_synchronous(L):
 
 def test_stream_status_without_ws(L):
     assert b.spa2_stream_status(None, None) == b.ERR_WORKSPACE
+
+
+def test_timing_symbols_without_a_gpu(L):
+    """The per-kernel timing aid: names for every kernel kind, and a read with
+    nothing recorded returns zero launches without touching a device."""
+    n = b.spa2_kernel_count()
+    names = [b.spa2_kernel_name(i) for i in range(n)]
+    assert len(set(names)) == n and "fwd_kernel" in names and "bwd_dkdv_kernel" in names
+    assert b.spa2_kernel_name(n) == "unknown"
+    assert b.spa2_timing_read() == {}
+    assert b.spa2_timing_enable(False) == b.OK

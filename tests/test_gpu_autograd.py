@@ -110,3 +110,39 @@ def test_velocity_distillation_steps_lower_the_loss():
         losses.append(loss.item())
     assert np.isfinite(losses).all()
     assert losses[-1] < 0.8 * losses[0], losses
+
+
+def test_forward_only_errors_are_raised():
+    """Inference without a backward: a V value outside the fp16 range is clamped
+    and recorded on the device; check_errors() raises it (no backward needed),
+    and later calls run clean."""
+    from trainable_block_sparse_pooled_b200.autograd import check_errors
+    q, k, v = synth.gaussian_with_sinks(B=1, H=1, N=384, d=64, seed=41, device="cuda")
+    check_errors()
+    bad = v.clone()
+    bad[0, 0, 5, 7] = 1e6
+    with torch.no_grad():
+        sparse_attention(q, k, bad, 0.3, 0.5)
+    with pytest.raises(b.Spa2Error) as e:
+        check_errors()
+    assert e.value.code == b.ERR_RANGE
+    with torch.no_grad():
+        o = sparse_attention(q, k, v, 0.3, 0.5)
+    check_errors()
+    assert torch.isfinite(o.float()).all()
+
+
+def test_workspaces_are_per_stream():
+    """The same shape on two streams gets two workspace sets."""
+    from trainable_block_sparse_pooled_b200 import autograd
+    q, k, v = synth.gaussian_with_sinks(B=1, H=1, N=256, d=64, seed=42, device="cuda")
+    side = torch.cuda.Stream()
+    o1 = sparse_attention(q, k, v, 0.3, 0.5)
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        o2 = sparse_attention(q, k, v, 0.3, 0.5)
+    torch.cuda.current_stream().wait_stream(side)
+    autograd.check_errors()
+    keys = [key for key in autograd._cache if key[:4] == (1, 1, 256, 64)]
+    assert len({key[-1] for key in keys}) == 2
+    assert torch.equal(o1, o2)

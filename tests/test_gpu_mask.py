@@ -14,9 +14,10 @@ from trainable_block_sparse_pooled_b200 import synth
 
 pytestmark = pytest.mark.gpu
 
-# P-bar (GPU fp32 vs oracle fp64): logits carry ~1e-6 relative error from fp32
-# pooling and dot products, which moves P-bar by that fraction of itself.
-PBAR_RTOL, PBAR_ATOL = 1e-4, 1e-6
+# P-bar (GPU fp32 vs oracle fp64): max-abs 1e-5 (P-bar <= 1). fp32 pooling and
+# dot products move a logit by ~1e-6 of its size, and P-bar moves by at most a
+# quarter of the logit error (dP/ds = P (1 - P) <= 1/4).
+PBAR_RTOL, PBAR_ATOL = 0.0, 1e-5
 
 
 def _mask_case(q, k, kf, pf):

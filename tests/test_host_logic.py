@@ -61,3 +61,25 @@ def test_calibration_bisection_property():
             assert pf == 0.0
 
     check()
+
+
+def test_bench_kept_flops_equals_oracle_attn_flops():
+    """bench.kept_flops (the numerator of every TFLOP/s figure) counts, from the
+    CSR form of a mask, what oracle.attn_flops counts from its dense form."""
+    import torch
+
+    import bench
+    from trainable_block_sparse_pooled_b200 import binding as b
+
+    rng = np.random.default_rng(3)
+    for N, bq, bkv in ((1000, 128, 64), (32760, 128, 64), (333, 128, 64), (5000, 256, 128), (700, 64, 128)):
+        Tm, Tn = oracle.block_counts(N, bq, bkv)
+        dense = rng.random((2, 3, Tm, Tn)) < 0.2
+        dense[..., rng.integers(Tn)] = True                       # no empty row
+        cnt = dense.sum(-1).astype(np.int32)
+        idx = np.full((2, 3, Tm, Tn), -1, dtype=np.int32)         # unused tail entries hold garbage
+        for pos in np.ndindex(cnt.shape):
+            ids = np.flatnonzero(dense[pos])
+            idx[pos][:ids.size] = ids
+        m = b.Mask(torch.tensor(cnt), torch.tensor(idx), None, None)
+        assert bench.kept_flops(m, N, 128, bq, bkv) == oracle.attn_flops(dense, N, bq, bkv, 128)

@@ -132,6 +132,23 @@ def test_attn_flops_counts_valid_rows_and_cols():
     assert oracle.attn_flops(mask, N, bq, bkv, d) == 4 * d * N * N
 
 
+@pytest.mark.parametrize("N,bq,bkv", [(1000, 128, 64), (333, 128, 64), (77, 64, 128), (2049, 256, 128)])
+def test_attn_flops_equals_brute_token_count(N, bq, bkv):
+    """Forward flops = 4 d per kept (query token, key token) pair: a random
+    ragged block mask expanded token by token and counted element by element."""
+    d = 128
+    Tm, Tn = oracle.block_counts(N, bq, bkv)
+    mask = _random_mask(N + bq, 2, 3, Tm, Tn, 0.3)
+    brute = sum(int(oracle.token_mask(mask[b, h], N, bq, bkv).sum()) for b in range(2) for h in range(3))
+    assert oracle.attn_flops(mask, N, bq, bkv, d) == 4.0 * d * brute
+    # a mask that differs in one block changes the count by that block's token pairs
+    m2 = mask.copy()
+    m2[0, 0, Tm - 1, Tn - 1] ^= True
+    rows, cols = N - (Tm - 1) * bq, N - (Tn - 1) * bkv
+    delta = 4.0 * d * rows * cols * (1 if m2[0, 0, Tm - 1, Tn - 1] else -1)
+    assert oracle.attn_flops(m2, N, bq, bkv, d) == oracle.attn_flops(mask, N, bq, bkv, d) + delta
+
+
 def test_sampled_backward_matches_full_backward():
     Q, K, V, dO = _inputs(11, N=450)
     B, H, N, d = Q.shape

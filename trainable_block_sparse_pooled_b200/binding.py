@@ -68,6 +68,10 @@ _SIGS = {
     "spa2_stream_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
     "spa2_debug_set_wait_limit_ns": (ctypes.c_int, [ctypes.c_longlong]),
     "spa2_debug_timeout_probe": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "spa2_timing_enable": (ctypes.c_int, [ctypes.c_int]),
+    "spa2_kernel_count": (ctypes.c_int, []),
+    "spa2_kernel_name": (ctypes.c_char_p, [ctypes.c_int]),
+    "spa2_timing_read": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_double)]),
 }
 
 
@@ -148,6 +152,28 @@ def spa2_debug_set_wait_limit_ns(limit: int) -> int:
 
 def spa2_debug_timeout_probe(ws, ws_bytes, stream) -> int:
     return lib().spa2_debug_timeout_probe(ws, ws_bytes, stream)
+
+
+def spa2_timing_enable(on: bool) -> int:
+    return lib().spa2_timing_enable(1 if on else 0)
+
+
+def spa2_kernel_count() -> int:
+    return lib().spa2_kernel_count()
+
+
+def spa2_kernel_name(kernel_id: int) -> str:
+    return lib().spa2_kernel_name(int(kernel_id)).decode()
+
+
+def spa2_timing_read() -> dict:
+    """{kernel name: (launches, summed event ms)} since the last read (kernels
+    with no launch omitted); waits for the recorded events."""
+    n = spa2_kernel_count()
+    launches = (ctypes.c_int * n)()
+    ms = (ctypes.c_double * n)()
+    _check(lib().spa2_timing_read(n, launches, ms), "spa2_timing_read")
+    return {spa2_kernel_name(i): (launches[i], ms[i]) for i in range(n) if launches[i]}
 
 
 # ---- torch conveniences -------------------------------------------------------

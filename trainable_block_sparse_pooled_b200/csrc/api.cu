@@ -6,6 +6,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -112,33 +114,68 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [BH, N, d] bf16 viewed as a 3-D tensor {d, N, BH}; box {64, rows, 1}, 128-byte
-// swizzle; rows past N of a head read as zero (no spill into the next head).
-static bool make_map(CUtensorMap* m, const void* ptr, const Shape& s, int rows, bool f16 = false) {
+enum MapType { MAP_BF16 = 0, MAP_F16 = 1, MAP_F32 = 2 };
+
+// Descriptor cache: a tensor map depends only on (address, shape, element
+// type, box rows), so the maps of buffers reused from call to call are encoded
+// once. Small, fixed size, round-robin replacement; guarded by a mutex.
+struct MapKey {
+  const void* ptr;
+  long long BH;
+  int N, d, rows, type;
+  bool operator==(const MapKey& o) const {
+    return ptr == o.ptr && BH == o.BH && N == o.N && d == o.d && rows == o.rows && type == o.type;
+  }
+};
+static constexpr int kMapCache = 64;
+static MapKey g_map_key[kMapCache];
+static CUtensorMap g_map_val[kMapCache];
+static bool g_map_used[kMapCache];
+static int g_map_next = 0;
+static std::mutex g_map_mu;
+
+// [BH, N, d] viewed as a 3-D tensor {d, N, BH}; box {64 bf16/fp16 or 32 fp32
+// columns (128 bytes), rows, 1}, 128-byte swizzle; rows past N of a head read
+// as zero (no spill into the next head) and are clipped on stores.
+static bool encode_map(CUtensorMap* m, const void* ptr, const Shape& s, int rows, int type) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
+  const cuuint64_t esz = type == MAP_F32 ? 4 : 2;
   cuuint64_t dims[3] = {(cuuint64_t)s.d, (cuuint64_t)s.N, (cuuint64_t)s.BH};
-  cuuint64_t strides[2] = {(cuuint64_t)s.d * 2, (cuuint64_t)s.N * s.d * 2};
-  cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+  cuuint64_t strides[2] = {(cuuint64_t)s.d * esz, (cuuint64_t)s.N * s.d * esz};
+  cuuint32_t box[3] = {type == MAP_F32 ? 32u : 64u, (cuuint32_t)rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUtensorMapDataType dt = type == MAP_F32   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                 : type == MAP_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                   : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUresult r = fn(m, dt, 3, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
-// [BH, N, d] fp32 tensor, box {32, rows, 1} (128 bytes wide), 128-byte swizzle
+static bool get_map(CUtensorMap* m, const void* ptr, const Shape& s, int rows, int type) {
+  const MapKey key{ptr, s.BH, s.N, s.d, rows, type};
+  std::lock_guard<std::mutex> lock(g_map_mu);
+  for (int i = 0; i < kMapCache; ++i)
+    if (g_map_used[i] && g_map_key[i] == key) {
+      *m = g_map_val[i];
+      return true;
+    }
+  if (!encode_map(m, ptr, s, rows, type)) return false;
+  const int slot = g_map_next;
+  g_map_next = (g_map_next + 1) % kMapCache;
+  g_map_key[slot] = key;
+  g_map_val[slot] = *m;
+  g_map_used[slot] = true;
+  return true;
+}
+
+static bool make_map(CUtensorMap* m, const void* ptr, const Shape& s, int rows, bool f16 = false) {
+  return get_map(m, ptr, s, rows, f16 ? MAP_F16 : MAP_BF16);
+}
+
 static bool make_map_f32(CUtensorMap* m, const void* ptr, const Shape& s, int rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)s.d, (cuuint64_t)s.N, (cuuint64_t)s.BH};
-  cuuint64_t strides[2] = {(cuuint64_t)s.d * 4, (cuuint64_t)s.N * s.d * 4};
-  cuuint32_t box[3] = {32, (cuuint32_t)rows, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  return get_map(m, ptr, s, rows, MAP_F32);
 }
 
 static int topk_count(float k_frac, int Tn) {
@@ -167,6 +204,7 @@ __global__ void timeout_probe_kernel(int* status, unsigned long long limit_ns) {
 }
 
 cudaError_t launch_timeout_probe(int* status, unsigned long long limit_ns, cudaStream_t s) {
+  KernelTimer kt(KID_PROBE, s);
   timeout_probe_kernel<<<1, 32, 0, s>>>(status, limit_ns);
   return cudaGetLastError();
 }

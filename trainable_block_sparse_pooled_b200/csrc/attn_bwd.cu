@@ -778,10 +778,13 @@ static cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
   const long long rows = (long long)a.BH * a.N;
   // 1. D and the fp16 copies of dO and V
   constexpr int PRE_ROWS = 256 / (D / 8);  // rows per 256-thread block
-  bwd_pre_kernel<D><<<(unsigned)((rows + PRE_ROWS - 1) / PRE_ROWS), 256, 0, s>>>(
+  {
+    KernelTimer kt(KID_BWD_PRE, s);
+    bwd_pre_kernel<D><<<(unsigned)((rows + PRE_ROWS - 1) / PRE_ROWS), 256, 0, s>>>(
       (const __nv_bfloat16*)a.o, (const __nv_bfloat16*)a.o_lo, (const __nv_bfloat16*)a.dout,
       (const __nv_bfloat16*)a.v, (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, a.dvec, (uint32_t*)a.do16,
       (uint32_t*)a.v16, (uint32_t*)a.q16, (uint32_t*)a.k16, rows, a.status);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // 2. dK, dV (kv-major)
@@ -789,6 +792,7 @@ static cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
     const size_t smem = sizeof(BwdSmem<D>) + 1024;
     e = cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    KernelTimer kt(KID_BWD_DKDV, s);
     bwd_dkdv_kernel<D><<<dim3(a.Tn, a.BH), BWD_THREADS, smem, s>>>(
         *a.tm_q16, *a.tm_k16, *a.tm_v, *a.tm_do, a.lse, a.dvec, a.col_cnt, a.col_idx, a.dk, a.dv, a.grad_f32, a.N, a.Tm,
         a.Tn, a.scale, a.scale_log2, a.status, a.wait_limit_ns);
@@ -800,6 +804,7 @@ static cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
     const size_t smem = sizeof(DqSmem<D>) + 1024;
     e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    KernelTimer kt(KID_BWD_DQ, s);
     bwd_dq_kernel<D><<<dim3(a.Tm, a.BH), DQ_THREADS, smem, s>>>(
         *a.tm_k, *a.tm_v, *a.tm_dq, static_cast<const __nv_bfloat16*>(a.q), static_cast<const __half*>(a.do16),
         a.lse, a.dvec, a.row_cnt, a.row_idx, a.grad_f32, a.N, a.Tm, a.Tn, a.scale, a.scale_log2, a.status,

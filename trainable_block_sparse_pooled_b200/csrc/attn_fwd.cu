@@ -342,12 +342,14 @@ __global__ void __launch_bounds__(256) v_to_f16_kernel(const uint4* __restrict__
 cudaError_t launch_v_to_f16(const void* v, void* v16, long long elems, int* status, cudaStream_t s) {
   const long long n8 = elems / 8;
   const unsigned blocks = (unsigned)((n8 + 255) / 256 < 148LL * 32 ? (n8 + 255) / 256 : 148LL * 32);
+  KernelTimer kt(KID_V16, s);
   v_to_f16_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4*>(v), static_cast<uint4*>(v16), n8, status);
   return cudaGetLastError();
 }
 
 cudaError_t launch_fwd(const FwdArgs& a, int d, cudaStream_t s) {
   dim3 grid(a.Tm, a.BH);
+  KernelTimer kt(KID_FWD, s);
   if (d == 128) {
     const size_t smem = sizeof(FwdSmem<128>) + 1024;
     cudaError_t e = cudaFuncSetAttribute(fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -7,6 +7,35 @@
 
 namespace spa2 {
 
+// timing.cu: per-kernel event timing (spa2_timing_*). One id per kernel kind.
+enum KernelId : int {
+  KID_POOL = 0,
+  KID_SELECT,
+  KID_CSC,
+  KID_PBAR_SELECT,
+  KID_V16,
+  KID_FWD,
+  KID_BWD_PRE,
+  KID_BWD_DKDV,
+  KID_BWD_DQ,
+  KID_PROBE,
+  KID_COUNT
+};
+
+// Brackets one kernel launch with two CUDA events recorded on `s` while timing
+// is on (construct it just before the launch, in the launch's scope).
+class KernelTimer {
+ public:
+  KernelTimer(int kid, cudaStream_t s);
+  ~KernelTimer();
+  KernelTimer(const KernelTimer&) = delete;
+  KernelTimer& operator=(const KernelTimer&) = delete;
+
+ private:
+  int slot_;
+  cudaStream_t s_;
+};
+
 struct MaskOut {
   int* row_cnt;
   int* row_idx;

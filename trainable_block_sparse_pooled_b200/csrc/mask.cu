@@ -386,6 +386,7 @@ static cudaError_t launch_select_t(const float* qbar, const float* kbar, int h0,
   const size_t smem = ((size_t)4 * KCH * D + (size_t)ROWS * D + (size_t)ROWS * 32 * E) * 4 + 4 * 8;
   cudaError_t e = cudaFuncSetAttribute(select_kernel<D, E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  KernelTimer kt(KID_SELECT, s);
   select_kernel<D, E><<<dim3((Tm + ROWS - 1) / ROWS, nh), 256, smem, s>>>(
       qbar, kbar, h0, Tm, Tn, W, 1.0f / sqrtf((float)D), K, thr, out, bits, status, wait_limit_ns);
   return cudaGetLastError();
@@ -407,18 +408,22 @@ cudaError_t launch_mask(const void* q, const void* k, float* qbar, float* kbar, 
                         int* col_idx, uint32_t* bits, int W, int* status, unsigned long long wait_limit_ns,
                         cudaStream_t s) {
   dim3 grid(Tm + Tn, BH);
+  {
+  KernelTimer kt(KID_POOL, s);
   if (d == 128)
     pool_kernel<128><<<grid, 256, 0, s>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qbar, kbar, 0, N, Tm, Tn,
                                           bq, bkv);
   else
     pool_kernel<64><<<grid, 256, 0, s>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qbar, kbar, 0, N, Tm, Tn,
                                          bq, bkv);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = (d == 128) ? launch_select_d<128>(qbar, kbar, 0, BH, Tm, Tn, W, K, thr, out, bits, status, wait_limit_ns, s)
                  : launch_select_d<64>(qbar, kbar, 0, BH, Tm, Tn, W, K, thr, out, bits, status, wait_limit_ns, s);
   if (e != cudaSuccess) return e;
   if (col_cnt) {
+    KernelTimer kt(KID_CSC, s);
     csc_kernel<<<dim3((Tn + 7) / 8, BH), 256, 0, s>>>(bits, 0, Tm, Tn, W, col_cnt, col_idx);
     e = cudaGetLastError();
   }
@@ -429,6 +434,7 @@ cudaError_t launch_select(const float* pbar, int BH, int Tm, int Tn, int K, unsi
                           const MaskOut& out, uint32_t* bits, int W, int* status, cudaStream_t s) {
   dim3 grid((Tm + 7) / 8, BH);
   const int e = (Tn + 31) / 32;
+  KernelTimer kt(KID_PBAR_SELECT, s);
   if (e <= 8)
     pbar_select_kernel<8><<<grid, 256, 0, s>>>(pbar, Tm, Tn, W, K, thr, out, bits, status);
   else if (e <= 16)
@@ -443,6 +449,7 @@ cudaError_t launch_select(const float* pbar, int BH, int Tm, int Tn, int K, unsi
 cudaError_t launch_csc(const uint32_t* bits, int BH, int Tm, int Tn, int W, int* col_cnt, int* col_idx,
                        cudaStream_t s) {
   dim3 grid((Tn + 7) / 8, BH);
+  KernelTimer kt(KID_CSC, s);
   csc_kernel<<<grid, 256, 0, s>>>(bits, 0, Tm, Tn, W, col_cnt, col_idx);
   return cudaGetLastError();
 }

@@ -12,7 +12,9 @@
 // Setup: on the first call on each device (with that device current), the
 // address of the array on that device is looked up once with
 // cudaGetSymbolAddress and cached; that lookup may load the module. Make the
-// first call on each device before any stream capture begins.
+// first call on each device before any stream capture begins. A
+// cudaDeviceReset unloads the module on that device, so the cached address is
+// stale afterwards: calls after a reset are not supported.
 //
 // Limits: one array per device, shared by every call on that device, so two
 // calls whose executions overlap (different streams, or different host
