@@ -60,7 +60,7 @@ def code_digest(path):
 
 
 KERNEL_SOURCES = {
-    "pool_kernel": "mask.cu", "select_kernel": "mask.cu", "csc_kernel": "mask.cu",
+    "pool_kernel": "mask.cu", "logits_kernel": "mask.cu", "select_kernel": "mask.cu", "csc_kernel": "mask.cu",
     "v_to_f16_kernel": "attn_fwd.cu", "fwd_kernel": "attn_fwd.cu",
     "bwd_pre_kernel": "attn_bwd.cu", "bwd_dkdv_kernel": "attn_bwd.cu", "bwd_dq_kernel": "attn_bwd.cu",
 }
@@ -118,11 +118,12 @@ def kernel_work(name, B, H, N, d, Tm, Tn, kept, fwd_flops):
         return "tensor", 2.0 * fwd_flops, "flop"
     if name == "bwd_dq_kernel":
         return "tensor", 0.5 * fwd_flops, "flop"
-    if name == "pool_kernel":
+    if name == "pool_kernel":     # Q and K read, Qbar and Kbar written
         return "hbm", 2.0 * e * 2 + 4.0 * B * H * (Tm + Tn) * d, "byte"
-    if name == "select_kernel":
-        return "hbm", 4.0 * B * H * (Tm + Tn) * d + 4.0 * (kept + B * H * Tm) + 4.0 * B * H * Tm * ((Tn + 31) // 32), \
-            "byte"
+    if name == "logits_kernel":   # Qbar and Kbar read, pooled logits written
+        return "hbm", 4.0 * B * H * (Tm + Tn) * d + 4.0 * B * H * Tm * Tn, "byte"
+    if name == "select_kernel":   # pooled logits read, CSR and kept-bit words written
+        return "hbm", 4.0 * B * H * Tm * Tn + 4.0 * (kept + B * H * Tm) + 4.0 * B * H * Tm * ((Tn + 31) // 32), "byte"
     if name == "csc_kernel":
         return "hbm", 4.0 * B * H * Tm * ((Tn + 31) // 32) + 4.0 * (kept + B * H * Tn), "byte"
     if name == "v_to_f16_kernel":
@@ -420,16 +421,27 @@ def run_gpu(args, wl, name):
     clocks.start()
     time.sleep(0.15)
     torch.cuda.nvtx.range_push("spa2_timed")     # ncu --nvtx-include "spa2_timed/" selects this region
-    b.spa2_timing_read()                         # forget launches recorded before the timed region
-    b.spa2_timing_enable(True)                   # per-kernel CUDA events on the launch stream
     t_start.record()
     for i in range(args.steps):
         step(evs[i])
     t_end.record()
     torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
+    # The same K steps again with a CUDA event pair around every kernel launch
+    # (spa2_timing_enable): per-kernel durations for `kernels` and `roofline`.
+    # Kept out of the headline steps above because an event between two kernels
+    # stops the second from starting early (programmatic dependent launch).
+    b.spa2_timing_read()
+    b.spa2_timing_enable(True)
+    p_start, p_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    p_start.record()
+    for i in range(args.steps):
+        step()
+    p_end.record()
+    torch.cuda.synchronize()
     b.spa2_timing_enable(False)
     per_kernel = b.spa2_timing_read()
+    profiled_ms = p_start.elapsed_time(p_end) / args.steps
     clk = clocks.stop()
     barrier(dist)
     s.check()
@@ -503,7 +515,7 @@ def run_gpu(args, wl, name):
     for kname, (n_launch, tot_ms) in per_kernel.items():
         bound, work, unit = kernel_work(kname, B, H, N, d, s.Tm, s.Tn, kept, fwd_flops)
         avg_ms = tot_ms / n_launch
-        ent = {"launches": n_launch, "avg_us": avg_ms * 1e3, "share": tot_ms / (ms * args.steps)}
+        ent = {"launches": n_launch, "avg_us": avg_ms * 1e3, "share": tot_ms / (profiled_ms * args.steps)}
         if bound == "tensor":
             ent.update(bound="tensor", achieved=work / (avg_ms * 1e-3) / 1e12, unit="TFLOP/s")
             ent["frac"] = ent["achieved"] / tensor_peak
@@ -534,6 +546,9 @@ def run_gpu(args, wl, name):
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": sum(v["launches"] for v in kernels.values()),
+        "kernel_timing": {"steps": args.steps, "ms_per_step": profiled_ms,
+                          "how": "the timed steps repeated with a CUDA event pair on the launch stream around each "
+                                 "kernel; avg_us = summed event time / launches; share = of that pass's step time"},
         "clocks": clk,
         "kernels": kernels,
         "ops": {"mask_us": mask_ms * 1e3, "mask_GBps": mask_gbs, "mask_hbm_frac": mask_gbs / pk["hbm_gbs"],

@@ -37,7 +37,7 @@ def test_workspace_sizes(L):
     B, H, N, d = 1, 12, 32760, 128
     Tm, Tn = 256, 512
     m = b.spa2_workspace_bytes(b.OP_MASK, B, H, N, d)
-    assert m >= 256 + B * H * (Tm + Tn) * d * 4 + B * H * Tm * 16 * 4
+    assert m >= 256 + B * H * (Tm + Tn) * d * 4 + B * H * Tm * 16 * 4   # Qbar, Kbar^T, kept-bit words
     assert b.spa2_workspace_bytes(b.OP_FWD, B, H, N, d) == 256 + B * H * N * d * 2   # status + fp16 V
     al = lambda n: -(-n // 256) * 256  # noqa: E731
     # status word, D (fp32 per row), fp16 copies of dO, V, Q and K, each 256-byte aligned

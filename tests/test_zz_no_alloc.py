@@ -68,7 +68,7 @@ def test_noalloc_ragged_shapes_in_a_row():
 
 def test_noalloc_refuses_oversize_shapes():
     """Scratch beyond the fixed size is refused before anything is launched."""
-    B, H, N, d = 1, 40, 131072, 128
+    B, H, N, d = 4, 40, 131072, 128
     need = b.spa2_workspace_bytes(b.OP_MASK, B, H, N, d)
     assert need > SCRATCH_BYTES
     dummy = ctypes.c_void_p(16)              # never dereferenced: the size check comes first

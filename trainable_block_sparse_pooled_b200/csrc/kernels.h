@@ -11,6 +11,7 @@ namespace spa2 {
 enum KernelId : int {
   KID_POOL = 0,
   KID_SELECT,
+  KID_LOGITS,
   KID_CSC,
   KID_PBAR_SELECT,
   KID_V16,
@@ -44,10 +45,13 @@ struct MaskOut {
 };
 
 // mask.cu
-cudaError_t launch_mask(const void* q, const void* k, float* qbar, float* kbar, int BH, int N, int d, int Tm, int Tn,
-                        int bq, int bkv, int K, unsigned long long thr, const MaskOut& out, int* col_cnt,
-                        int* col_idx, uint32_t* bits, int W, int* status, unsigned long long wait_limit_ns,
-                        cudaStream_t s);
+// qbar: Qbar workspace [BH, Tm, d] fp32; kbT: Kbar^T workspace [BH, d, kbar_cols(Tn)] fp32;
+// lg: logit workspace [BH, Tm, Tn] fp32
+int kbar_cols(int Tn);
+cudaError_t launch_mask(const void* q, const void* k, float* qbar, float* kbT, float* lg, int BH, int N, int d,
+                        int Tm, int Tn, int bq, int bkv, int K, unsigned long long thr, const MaskOut& out,
+                        int* col_cnt, int* col_idx, uint32_t* bits, int W, int* status,
+                        unsigned long long wait_limit_ns, cudaStream_t s);
 cudaError_t launch_select(const float* pbar, int BH, int Tm, int Tn, int K, unsigned long long thr,
                           const MaskOut& out, uint32_t* bits, int W, int* status, cudaStream_t s);
 cudaError_t launch_csc(const uint32_t* bits, int BH, int Tm, int Tn, int W, int* col_cnt, int* col_idx,

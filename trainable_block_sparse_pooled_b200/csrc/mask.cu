@@ -1,14 +1,23 @@
 // Block-mask kernels: steps 1-3 of SpargeAttention2 (paper.rainbus.top summary,
 // 方法步骤详情 steps 1-3; 技术新颖性 union formula; gist.science 2A).
 //
-//   pool_kernel    one CTA per block: mean of each q-block (b_q rows) and kv-block
-//                  (b_kv rows) of Q / K -> Qbar [B,H,Tm,d], Kbar [B,H,Tn,d] fp32.
-//   select_kernel  8 q-block rows of one head per CTA, one warp per row: fp32
-//                  logits against Kbar (streamed through a 4-deep smem ring with
-//                  bulk async copies), softmax -> P-bar, hybrid selection -> CSR,
-//                  kept-bit words, optional P-bar / uint8 bitmap.
-//   csc_kernel     kept-bit words -> CSC, one warp per kv-block column.
+//   pool_kernel    one CTA per block, every streaming load of a thread in flight
+//                  before it sums: means of the q-blocks -> Qbar
+//                  [B*H, T_m, d] and of the kv-blocks -> Kbar^T [B*H, d, T_n']
+//                  fp32 (transposed, T_n' = T_n rounded up to a multiple of 4,
+//                  so the logit loop reads the keys of one feature with
+//                  coalesced 8-byte loads).
+//   logits_kernel  S-bar = Qbar Kbar^T / sqrt(d), fp32, by CTAs of 16 rows x 128
+//                  keys of one head (thread = pair of keys against 4 rows) ->
+//                  logit scratch [B*H, T_m, T_n].
+//   select_kernel  one warp per row, the row in registers: softmax -> P-bar,
+//                  hybrid selection -> CSR, kept-bit words, optional P-bar /
+//                  uint8 bitmap.
+//   csc_kernel     kept-bit words -> CSC: one CTA per (head, 32-column word),
+//                  32x32 bit transposes with warp ballots.
 //   pbar_select_kernel  the selection alone on a caller-given P-bar.
+// The four mask kernels run back to back on one stream; each after the first is
+// launched as a programmatic dependent of the one before.
 //
 // Selection is exact integer work on the float32 P-bar: ranks are (value desc,
 // id asc); Top-k keeps the first K ranks; Top-p keeps rank r while the
@@ -17,7 +26,13 @@
 // ranks, and the value at rank n-1 is the largest key T with
 //   count(key >= T) >= K  and  mass(key >= T) >= thr,
 // found by one bisection over the float bit patterns (monotone for P >= 0),
-// with ties at T taken by ascending block id. No sort, no atomics. Each lane
+// with ties at T taken by ascending block id. No sort, no atomics. Rows that
+// keep at most 64 blocks are instead walked rank by rank (extract_top), the
+// warp taking the largest key of per-lane top-4 caches at each step. The
+// bisection passes over the whole row only until at most 32 keys remain
+// between its bounds; those are compacted to one per lane and the rest of the
+// search counts them with ballots (keys above the bracket are carried as a
+// count and a mass, keys below it never count). Each lane
 // keeps its E = ceil(T_n / 32) keys and masses in registers; masses are split
 // as q >> 16 and q & 0xffff so warp sums stay exact in 32 bits
 // (__reduce_add_sync) for rows of fewer than 2^15 blocks.
@@ -29,50 +44,9 @@ namespace spa2 {
 namespace {
 
 constexpr int ROWS = 8;  // P-bar rows per select CTA (one warp each)
-constexpr int KCH = 32;  // Kbar rows per staged chunk
 
 SPA2_DEV unsigned long long mass_of(float p) {
   return __float2ull_rz(p * 4294967296.0f);  // exact: power-of-two scale of p in [0, 1]
-}
-
-// ---------------------------------------------------------------------------
-// pooling of one block: 16-byte streaming loads, all rows of a thread in flight
-// ---------------------------------------------------------------------------
-template <int D>
-SPA2_DEV void pool_block(const __nv_bfloat16* __restrict__ src, int rows, float* __restrict__ dst, float* red) {
-  constexpr int TPR = D / 8;     // threads per row (8 bf16 each)
-  constexpr int RP = 256 / TPR;  // rows per pass
-  constexpr int MAXIT = 128 / RP;
-  const int tr = threadIdx.x / TPR, tc = threadIdx.x % TPR;
-  float acc[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-  const uint4* base = reinterpret_cast<const uint4*>(src) + tc;
-  uint4 v[MAXIT];
-#pragma unroll
-  for (int u = 0; u < MAXIT; ++u) {
-    const int r = tr + u * RP;
-    v[u] = (r < rows) ? __ldcs(base + (long long)r * TPR) : make_uint4(0, 0, 0, 0);
-  }
-#pragma unroll
-  for (int u = 0; u < MAXIT; ++u) {
-    const __nv_bfloat162* hp = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 f = __bfloat1622float2(hp[e]);
-      acc[2 * e] += f.x;
-      acc[2 * e + 1] += f.y;
-    }
-  }
-#pragma unroll
-  for (int e = 0; e < 8; ++e) red[tr * (D + 1) + tc * 8 + e] = acc[e];
-  __syncthreads();
-  if (threadIdx.x < D) {
-    float s = 0.f;
-#pragma unroll 8
-    for (int i = 0; i < RP; ++i) s += red[i * (D + 1) + threadIdx.x];
-    dst[threadIdx.x] = s / static_cast<float>(rows);
-  }
 }
 
 // ---------------------------------------------------------------------------
@@ -80,11 +54,138 @@ SPA2_DEV void pool_block(const __nv_bfloat16* __restrict__ src, int rows, float*
 // e < E, of the row: key = float bits of P-bar (0 for padding), mh / ml = mass
 // halves (0 for padding)
 // ---------------------------------------------------------------------------
+// Kept ids of a row from its kept-bit words (bal[e] bit l = element 32 e + l):
+// CSR row in ascending order, kept-bit words, optional uint8 bitmap; checks the
+// count against n.
 template <int E>
-SPA2_DEV void select_row_regs(const uint32_t (&key)[E], const uint32_t (&mh)[E], const uint32_t (&ml)[E], int Tn,
-                              int K, unsigned long long thr, int* row_cnt_out, int* row_idx_out, uint32_t* bits_out,
-                              uint8_t* bitmap_out, int* status) {
+SPA2_DEV void emit_row(const uint32_t (&bal)[E], int Tn, int n, int* row_cnt_out, int* row_idx_out,
+                       uint32_t* bits_out, uint8_t* bitmap_out, int* status) {
   const uint32_t lane = lane_id();
+  const uint32_t lt = (1u << lane) - 1u;
+  int running = 0;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int j = 32 * e + (int)lane;
+    if (32 * e < Tn) {
+      const bool keep = (bal[e] >> lane) & 1u;
+      if (keep) row_idx_out[running + __popc(bal[e] & lt)] = j;
+      if (bitmap_out && j < Tn) bitmap_out[j] = keep ? 1 : 0;
+      if (lane == 0) bits_out[e] = bal[e];
+      running += __popc(bal[e]);
+    }
+  }
+  if (lane == 0) {
+    *row_cnt_out = running;
+    if (running != n) report(status, SPA2_ERR_DEVICE_BOUNDS);
+  }
+}
+
+// Exact rank-order walk for rows that keep few blocks. Ranks are taken one at a
+// time as the warp maximum of (key desc, id asc): every lane keeps its own
+// best 4 not-yet-taken elements in a sorted cache of packed 64-bit values
+// (refilled from its registers when it runs dry), the warp takes the largest cached key (REDUX max) and,
+// among lanes holding that key, the lowest block id (REDUX min). Rank r is kept
+// while r < K or the mass of ranks < r is below thr, exactly the rule of the
+// bisection below. Returns false, having changed nothing, when the row keeps
+// more than EXTRACT_CAP ranks; otherwise kept = this lane's kept elements (bit
+// e = element lane + 32 e) and n = their count over the warp.
+constexpr int EXTRACT_CAP = 64;
+
+// This lane's best 4 elements not yet taken, as packed 64-bit values
+// ((key + 1) << 8 | (255 - e)): a larger value is a higher rank (larger key,
+// then smaller e); 0 marks an empty slot. Kept sorted, hk[0] the best.
+template <int E>
+SPA2_DEV void top4_refill(const uint32_t (&key)[E], int Tn, uint64_t taken, uint64_t (&hk)[4]) {
+  const uint32_t lane = lane_id();
+#pragma unroll
+  for (int j = 0; j < 4; ++j) hk[j] = 0ull;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    uint64_t v = ((int)lane + 32 * e < Tn && !((taken >> e) & 1ull))
+                     ? ((uint64_t)(key[e] + 1u) << 8) | (uint64_t)(255 - e)
+                     : 0ull;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {  // insertion by compare-exchange
+      const uint64_t hi = v > hk[j] ? v : hk[j];
+      v = v > hk[j] ? hk[j] : v;
+      hk[j] = hi;
+    }
+  }
+}
+
+template <int E>
+SPA2_DEV bool extract_top(const uint32_t (&key)[E], int Tn, int K, unsigned long long thr, uint64_t& kept,
+                          int& n_out) {
+  const uint32_t lane = lane_id();
+  uint64_t hk[4];
+  kept = 0ull;
+  top4_refill<E>(key, Tn, kept, hk);
+  int mine = 0;  // valid elements of this lane not yet taken
+#pragma unroll
+  for (int e = 0; e < E; ++e) mine += ((int)lane + 32 * e < Tn) ? 1 : 0;
+  unsigned long long before = 0ull;  // mass of the ranks taken so far
+  for (int r = 0; r <= EXTRACT_CAP; ++r) {
+    if (r == Tn) {  // every block taken
+      n_out = r;
+      return true;
+    }
+    if (hk[0] == 0ull && mine > 0) top4_refill<E>(key, Tn, kept, hk);
+    const uint32_t hkey = (uint32_t)(hk[0] >> 8);  // key + 1, or 0
+    const uint32_t gmax = __reduce_max_sync(0xffffffff, hkey);
+    const uint32_t id = (hkey == gmax) ? lane + 32u * (255u - (uint32_t)(hk[0] & 255u)) : 0xFFFFFFFFu;
+    const uint32_t wid = __reduce_min_sync(0xffffffff, id);
+    if (!(r < K || before < thr)) {  // rank r is the first one dropped
+      n_out = r;
+      return true;
+    }
+    if (r == EXTRACT_CAP) break;
+    before += mass_of(__uint_as_float(gmax - 1u));
+    if (lane == (wid & 31u)) {
+      kept |= 1ull << (wid >> 5);
+      --mine;
+      hk[0] = hk[1];
+      hk[1] = hk[2];
+      hk[2] = hk[3];
+      hk[3] = 0ull;
+    }
+  }
+  kept = 0ull;
+  return false;
+}
+
+template <int E>
+SPA2_DEV uint32_t eq_all_ties(const uint32_t (&key)[E], uint32_t bv, int Tn) {
+  uint32_t eq = 0u;
+#pragma unroll
+  for (int e = 0; e < E; ++e) eq += ((int)lane_id() + 32 * e < Tn && key[e] == bv) ? 1u : 0u;
+  return __reduce_add_sync(0xffffffff, eq);
+}
+
+template <int E>
+SPA2_DEV void select_row_regs(const uint32_t (&key)[E], int Tn, int K, unsigned long long thr, int* row_cnt_out,
+                              int* row_idx_out, uint32_t* bits_out, uint8_t* bitmap_out, int* status,
+                              uint32_t* scratch /* 96 words, this warp's */) {
+  const uint32_t lane = lane_id();
+  const uint32_t lt = (1u << lane) - 1u;
+  uint32_t bal[E];
+  if (K < Tn && K <= EXTRACT_CAP) {
+    uint64_t kept;
+    int n_kept;
+    if (extract_top<E>(key, Tn, K, thr, kept, n_kept)) {
+#pragma unroll
+      for (int e = 0; e < E; ++e) bal[e] = __ballot_sync(0xffffffff, (kept >> e) & 1ull);
+      emit_row<E>(bal, Tn, n_kept, row_cnt_out, row_idx_out, bits_out, bitmap_out, status);
+      return;
+    }
+  }
+  // bisection path: quantised masses, split into 16-bit halves
+  uint32_t mh[E], ml[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const unsigned long long q = mass_of(__uint_as_float(key[e]));  // padding keys are 0: mass 0
+    mh[e] = (uint32_t)(q >> 16);
+    ml[e] = (uint32_t)(q & 0xffffull);
+  }
   uint32_t kmin = 0xFFFFFFFFu, kmax = 0u, th = 0u, tl = 0u;
 #pragma unroll
   for (int e = 0; e < E; ++e) {
@@ -105,14 +206,20 @@ SPA2_DEV void select_row_regs(const uint32_t (&key)[E], const uint32_t (&mh)[E],
   if (!keep_all) {
     // largest T with count(key >= T) >= K and mass(key >= T) >= thr; T = kmin satisfies
     // both (count Tn >= K, mass = total >= thr), T = kmax + 1 satisfies neither
+    // Every mid tested is > lo >= 0, so padding keys (0) never count. cnt_lo /
+    // cnt_hi are the numbers of valid keys >= lo / >= hi, m_hi the mass of the
+    // keys >= hi; keys in [lo, hi) are the only ones the remaining tests can split.
     uint32_t lo = kmin, hi = kmax + 1u;
+    uint32_t cnt_lo = (uint32_t)Tn, cnt_hi = 0u;
+    unsigned long long m_hi = 0ull;
+    // phase A: passes over the whole row until at most 32 keys lie in [lo, hi)
 #pragma unroll 1
-    while (hi - lo > 1u) {
+    while (hi - lo > 1u && cnt_lo - cnt_hi > 32u) {
       const uint32_t mid = lo + ((hi - lo) >> 1);
       uint32_t c = 0u, sh = 0u, sl = 0u;
 #pragma unroll
       for (int e = 0; e < E; ++e) {
-        const bool in = key[e] >= mid;  // padding keys are 0 < mid
+        const bool in = key[e] >= mid;
         c += in ? 1u : 0u;
         sh += in ? mh[e] : 0u;
         sl += in ? ml[e] : 0u;
@@ -120,7 +227,50 @@ SPA2_DEV void select_row_regs(const uint32_t (&key)[E], const uint32_t (&mh)[E],
       c = __reduce_add_sync(0xffffffff, c);
       const unsigned long long mass =
           ((unsigned long long)__reduce_add_sync(0xffffffff, sh) << 16) + __reduce_add_sync(0xffffffff, sl);
-      if (c >= (uint32_t)K && mass >= thr) lo = mid; else hi = mid;
+      if (c >= (uint32_t)K && mass >= thr) {
+        lo = mid;
+        cnt_lo = c;
+      } else {
+        hi = mid;
+        cnt_hi = c;
+        m_hi = mass;
+      }
+    }
+    // phase B: the <= 32 keys in [lo, hi) compacted to one per lane; keys >= hi
+    // enter through cnt_hi / m_hi, keys < lo never count
+    if (hi - lo > 1u) {
+      uint32_t base = 0u;
+      const uint32_t below = (1u << lane) - 1u;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const bool cand = ((int)lane + 32 * e < Tn) && key[e] >= lo && key[e] < hi;
+        const uint32_t bal = __ballot_sync(0xffffffff, cand);
+        if (cand) {
+          const uint32_t pos = base + __popc(bal & below);
+          scratch[pos] = key[e];
+          scratch[32 + pos] = mh[e];
+          scratch[64 + pos] = ml[e];
+        }
+        base += __popc(bal);
+      }
+      __syncwarp();
+      // Each lane counts the candidates >= its own key (itself and ties included):
+      // count(key >= own) = cnt_hi + that, and likewise the mass. The largest
+      // candidate key meeting both bounds is the answer; with none, lo is.
+      const bool have = lane < base;
+      const uint32_t own = have ? scratch[lane] : 0u;
+      uint32_t cge = 0u, sh = 0u, sl = 0u;
+#pragma unroll 4
+      for (uint32_t t = 0; t < base; ++t) {
+        const bool ge = scratch[t] >= own;
+        cge += ge ? 1u : 0u;
+        sh += ge ? scratch[32 + t] : 0u;
+        sl += ge ? scratch[64 + t] : 0u;
+      }
+      __syncwarp();
+      const unsigned long long mass = m_hi + ((unsigned long long)sh << 16) + sl;
+      const bool meets = have && cnt_hi + cge >= (uint32_t)K && mass >= thr;
+      lo = max(lo, __reduce_max_sync(0xffffffff, meets ? own : 0u));
     }
     uint32_t gt = 0u, eq = 0u, gh = 0u, gl = 0u;
 #pragma unroll
@@ -139,8 +289,13 @@ SPA2_DEV void select_row_regs(const uint32_t (&key)[E], const uint32_t (&mh)[E],
     const uint32_t tK = ((uint32_t)K > gt) ? (uint32_t)K - gt : 0u;
     uint32_t tR = 0u;
     if (thr > gm) {
+      // ceil((thr - gm) / qv) ties, at most eq: a double quotient (both operands
+      // < 2^34, so it is within one of the exact one) corrected in integers
       const unsigned long long qv = mass_of(__uint_as_float(lo));  // > 0: mass(key >= T) > mass(key > T)
-      const unsigned long long need = (thr - gm + qv - 1ull) / qv;
+      const unsigned long long rem = thr - gm;
+      unsigned long long need = (unsigned long long)ceil((double)rem / (double)qv);
+      if (need > 0ull && (need - 1ull) * qv >= rem) --need;
+      if (need * qv < rem) ++need;
       tR = (uint32_t)(need < (unsigned long long)eq ? need : (unsigned long long)eq);
     }
     bv = lo;
@@ -149,208 +304,264 @@ SPA2_DEV void select_row_regs(const uint32_t (&key)[E], const uint32_t (&mh)[E],
     keep_all = (n >= Tn);
   }
   // emit ascending ids: key > bv, or key == bv among the first bt by id
-  const uint32_t lt = (1u << lane) - 1u;
-  int running = 0;
-  uint32_t ties_seen = 0;
+  if (keep_all || bt == 0u || bt >= eq_all_ties(key, bv, Tn)) {
+    // no tie needs ranking: every tie at bv is kept (bt >= their count) or none is
+    const bool ties_in = !keep_all && bt != 0u;
 #pragma unroll
-  for (int e = 0; e < E; ++e) {
-    if (32 * e >= Tn) break;
-    const int j = 32 * e + (int)lane;
-    const bool valid = j < Tn;
-    const uint32_t u = key[e];
-    const bool is_tie = valid && (u == bv);
-    const uint32_t tie_bal = __ballot_sync(0xffffffff, is_tie);
-    const uint32_t tie_rank = ties_seen + __popc(tie_bal & lt);
-    const bool keep = valid && (keep_all || u > bv || (is_tie && tie_rank < bt));
-    const uint32_t bal = __ballot_sync(0xffffffff, keep);
-    if (keep) row_idx_out[running + __popc(bal & lt)] = j;
-    if (bitmap_out && valid) bitmap_out[j] = keep ? 1 : 0;
-    if (lane == 0) bits_out[e] = bal;
-    running += __popc(bal);
-    ties_seen += __popc(tie_bal);
+    for (int e = 0; e < E; ++e) {
+      const bool valid = (int)lane + 32 * e < Tn;
+      bal[e] = __ballot_sync(0xffffffff, valid && (keep_all || key[e] > bv || (ties_in && key[e] == bv)));
+    }
+  } else {
+    uint32_t ties_seen = 0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const bool valid = (int)lane + 32 * e < Tn;
+      const bool is_tie = valid && (key[e] == bv);
+      const uint32_t tie_bal = __ballot_sync(0xffffffff, is_tie);
+      const uint32_t tie_rank = ties_seen + __popc(tie_bal & lt);
+      bal[e] = __ballot_sync(0xffffffff, valid && (key[e] > bv || (is_tie && tie_rank < bt)));
+      ties_seen += __popc(tie_bal);
+    }
   }
-  if (lane == 0) {
-    *row_cnt_out = running;
-    if (running != n) report(status, SPA2_ERR_DEVICE_BOUNDS);
-  }
+  emit_row<E>(bal, Tn, n, row_cnt_out, row_idx_out, bits_out, bitmap_out, status);
 }
 
 // load a P-bar row (smem or global, length Tn) into lane registers and select
 template <int E>
 SPA2_DEV void select_row(const float* row, int Tn, int K, unsigned long long thr, int* row_cnt_out,
-                         int* row_idx_out, uint32_t* bits_out, uint8_t* bitmap_out, int* status) {
-  uint32_t key[E], mh[E], ml[E];
+                         int* row_idx_out, uint32_t* bits_out, uint8_t* bitmap_out, int* status, uint32_t* scratch) {
+  uint32_t key[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) {
     const int j = (int)lane_id() + 32 * e;
-    const float p = j < Tn ? row[j] : 0.f;
-    const unsigned long long q = mass_of(p);
-    key[e] = __float_as_uint(p);
-    mh[e] = (uint32_t)(q >> 16);
-    ml[e] = (uint32_t)(q & 0xffffull);
+    key[e] = __float_as_uint(j < Tn ? row[j] : 0.f);
   }
-  select_row_regs<E>(key, mh, ml, Tn, K, thr, row_cnt_out, row_idx_out, bits_out, bitmap_out, status);
+  select_row_regs<E>(key, Tn, K, thr, row_cnt_out, row_idx_out, bits_out, bitmap_out, status, scratch);
 }
 
-// CSC of one kv-block column c by one warp (ascending q-block ids)
-SPA2_DEV void csc_column_warp(const uint32_t* __restrict__ head_bits, int Tm, int W, int c, int* col_cnt_out,
-                              int* col_idx_out) {
-  const uint32_t lane = lane_id();
-  const uint32_t lt = (1u << lane) - 1u;
-  const uint32_t* col = head_bits + (c >> 5);
-  int running = 0;
-  for (int base = 0; base < Tm; base += 32 * 8) {
-    uint32_t w8[8];
+
+// softmax of one logit row (length Tn, already scaled by 1/sqrt(d)) and its
+// selection, by one warp with the row in lane registers: P = exp2((x - max)
+// log2 e) / sum, the sum inverted once; P-bar written to pbar_out when it is
+// not NULL
+template <int E>
+SPA2_DEV void softmax_select_row(const float* __restrict__ lrow, int Tn, int K, unsigned long long thr,
+                                 float* pbar_out, int* row_cnt_out, int* row_idx_out, uint32_t* bits_out,
+                                 uint8_t* bitmap_out, int* status, uint32_t* scratch) {
+  constexpr float LOG2E = 1.4426950408889634f;
+  const int lane = (int)lane_id();
+  float x[E];
+  float mx = -INFINITY;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {  // all loads of 8 row groups in flight
-      const int i = base + 32 * u + (int)lane;
-      w8[u] = (i < Tm) ? col[(long long)i * W] : 0u;
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = base + 32 * u + (int)lane;
-      const bool bit = (w8[u] >> (c & 31)) & 1u;
-      const uint32_t bal = __ballot_sync(0xffffffff, bit);
-      if (bit) col_idx_out[running + __popc(bal & lt)] = i;
-      running += __popc(bal);
-    }
+  for (int e = 0; e < E; ++e) {
+    const int j = lane + 32 * e;
+    x[e] = j < Tn ? lrow[j] : -INFINITY;
   }
-  if (lane == 0) *col_cnt_out = running;
+#pragma unroll
+  for (int e = 0; e < E; ++e) mx = fmaxf(mx, x[e]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffff, mx, o));
+  const float nm = -mx * LOG2E;
+  float ssum = 0.f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    x[e] = fast_exp2(fmaf(x[e], LOG2E, nm));  // 0 for padding (exp2(-inf))
+    ssum += x[e];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ssum += __shfl_xor_sync(0xffffffff, ssum, o);
+  const float inv = 1.0f / ssum;
+  uint32_t key[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int j = lane + 32 * e;
+    const float p = j < Tn ? x[e] * inv : 0.f;
+    if (pbar_out && j < Tn) pbar_out[j] = p;
+    key[e] = __float_as_uint(p);
+  }
+  select_row_regs<E>(key, Tn, K, thr, row_cnt_out, row_idx_out, bits_out, bitmap_out, status, scratch);
+}
+
+// CSC of 32 kv-block columns (one kept-bit word w of every row) of one head:
+// for each tile of 32 q-block rows a warp transposes the 32x32 bit block with
+// ballots (lane b then holds the bits of column 32w+b over the tile's rows),
+// counts are scanned across the tiles in shared memory, and every lane writes
+// the ascending row ids of its column.
+SPA2_DEV void csc_word_cta(const uint32_t* __restrict__ head_bits, int Tm, int Tn, int W, int w,
+                           int* __restrict__ col_cnt, int* __restrict__ col_idx, int* cnt_smem /* [8][32] */,
+                           int* base_smem /* [32] */) {
+  const int warp = threadIdx.x >> 5;
+  const int lane = (int)lane_id();
+  const int col = w * 32 + lane;
+  if (threadIdx.x < 32) base_smem[lane] = 0;
+  __syncthreads();
+  for (int t0 = 0; t0 < Tm; t0 += 8 * 32) {  // 8 row tiles of 32 per pass, one per warp
+    const int r0 = t0 + warp * 32;
+    const int row = r0 + lane;
+    const uint32_t word = row < Tm ? head_bits[(long long)row * W + w] : 0u;
+    uint32_t mine = 0u;
+#pragma unroll
+    for (int b = 0; b < 32; ++b) {
+      const uint32_t v = __ballot_sync(0xffffffffu, (word >> b) & 1u);
+      if (lane == b) mine = v;
+    }
+    cnt_smem[warp * 32 + lane] = __popc(mine);
+    __syncthreads();
+    int pos = base_smem[lane];
+    for (int u = 0; u < warp; ++u) pos += cnt_smem[u * 32 + lane];
+    if (col < Tn) {
+      int* dst = col_idx + (long long)col * Tm + pos;
+      while (mine) {
+        const int bit = __ffs(mine) - 1;
+        mine &= mine - 1u;
+        *dst++ = r0 + bit;
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      int tot = 0;
+      for (int u = 0; u < 8; ++u) tot += cnt_smem[u * 32 + lane];
+      base_smem[lane] += tot;
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x < 32 && col < Tn) col_cnt[col] = base_smem[lane];
 }
 
 }  // namespace
 
+// Pooling: one CTA of 256 threads per block (blockIdx.x < T_m: q-block ->
+// Qbar row-major; otherwise kv-block -> Kbar^T column). Each thread owns a
+// 16-byte column chunk of every 16th (d = 128) or 32nd (d = 64) row and issues
+// all of its streaming loads of a 128-row span before summing; partial sums
+// meet in shared memory.
 template <int D>
 __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ q,
                                                    const __nv_bfloat16* __restrict__ k, float* __restrict__ qbar,
-                                                   float* __restrict__ kbar, int h0, int N, int Tm, int Tn, int bq,
+                                                   float* __restrict__ kbT, int N, int Tm, int Tn, int TnP, int bq,
                                                    int bkv) {
-  __shared__ float red[(256 / (D / 8)) * (D + 1)];
+  constexpr int TPR = D / 8;        // threads per row (8 bf16 each)
+  constexpr int RP = 256 / TPR;     // rows per pass
+  constexpr int MAXIT = 128 / RP;   // loads per thread per 128-row span
+  __shared__ float red[RP * (D + 1)];
+  pdl_trigger();  // the select kernel may be scheduled; it waits for this grid before reading
   const int blk = blockIdx.x;
-  const long long h = h0 + blockIdx.y;
-  const __nv_bfloat16* src;
-  float* dst;
-  int rows;
-  if (blk < Tm) {
-    src = q + (h * N + (long long)blk * bq) * D;
-    rows = min(bq, N - blk * bq);
-    dst = qbar + (h * Tm + blk) * D;
-  } else {
-    const int j = blk - Tm;
-    src = k + (h * N + (long long)j * bkv) * D;
-    rows = min(bkv, N - j * bkv);
-    dst = kbar + (h * Tn + j) * D;
+  const long long h = blockIdx.y;
+  const bool is_q = blk < Tm;
+  const int idx = is_q ? blk : blk - Tm;
+  const int bsz = is_q ? bq : bkv;
+  const int rows = min(bsz, N - idx * bsz);
+  const __nv_bfloat16* src = (is_q ? q : k) + (h * N + (long long)idx * bsz) * D;
+  const int tr = threadIdx.x / TPR, tc = threadIdx.x % TPR;
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  const uint4* base = reinterpret_cast<const uint4*>(src) + tc;
+  for (int r0 = 0; r0 < rows; r0 += 128) {
+    uint4 v[MAXIT];
+#pragma unroll
+    for (int u = 0; u < MAXIT; ++u) {
+      const int r = r0 + tr + u * RP;
+      v[u] = (r < rows) ? __ldcs(base + (long long)r * TPR) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < MAXIT; ++u) {
+      const __nv_bfloat162* hp = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(hp[e]);
+        acc[2 * e] += f.x;
+        acc[2 * e + 1] += f.y;
+      }
+    }
   }
-  pool_block<D>(src, rows, dst, red);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) red[tr * (D + 1) + tc * 8 + e] = acc[e];
+  __syncthreads();
+  if (threadIdx.x < D) {
+    float sum = 0.f;
+#pragma unroll 8
+    for (int i = 0; i < RP; ++i) sum += red[i * (D + 1) + threadIdx.x];
+    const float mean = sum / static_cast<float>(rows);
+    if (is_q)
+      qbar[(h * Tm + idx) * D + threadIdx.x] = mean;
+    else
+      kbT[(h * D + threadIdx.x) * TnP + idx] = mean;
+  }
 }
 
-// 8 rows (one per warp) of head h0 + blockIdx.y: logits, softmax, selection
-template <int D, int E>
-__global__ void __launch_bounds__(256, (E <= 16 ? 2 : 1)) select_kernel(const float* __restrict__ qbar,
-                                                        const float* __restrict__ kbar, int h0, int Tm, int Tn, int W,
-                                                        float inv_sqrt_d, int K, unsigned long long thr, MaskOut out,
-                                                        uint32_t* __restrict__ bits, int* status,
-                                                        unsigned long long wait_limit_ns) {
-  constexpr int NST = 4;                                   // ring depth
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  float* ring = reinterpret_cast<float*>(smem_raw);        // [NST][KCH][D], unpadded
-  float* qb = ring + NST * KCH * D;                        // [ROWS][D]
-  float* lrows = qb + ROWS * D;                            // [ROWS][32 E]
-  uint64_t* full = reinterpret_cast<uint64_t*>(lrows + ROWS * 32 * E);  // [NST]
-  __shared__ int abort_flag;
-  const int warp = threadIdx.x >> 5;
-  const uint32_t lane = lane_id();
-  const long long h = h0 + blockIdx.y;
-  const int i0 = blockIdx.x * ROWS;
-  const float* kb = kbar + h * Tn * D;
-  const int nch = (Tn + KCH - 1) / KCH;
-  if (threadIdx.x == 0) {
-    for (int st = 0; st < NST; ++st) mbar_init(&full[st], 1);
-    abort_flag = 0;
-    fence_mbar_init();
+// Pooled logits: S-bar = Qbar Kbar^T / sqrt(d) -> lg [B*H, Tm, Tn] fp32. CTA
+// (key block of 128, row group of 16, head): the 16 pooled rows go to shared
+// memory transposed ([d][16]); thread (key pair kp, quarter hq) accumulates
+// keys 2kp, 2kp+1 against rows 4hq .. 4hq+3, the keys read from Kbar^T with
+// coalesced 8-byte loads (the four quarters of a CTA read the same keys, the
+// later ones from L1), 16 in flight.
+constexpr int LG_ROWS = 16, LG_KEYS = 128;
+
+template <int D>
+__global__ void __launch_bounds__(256) logits_kernel(const float* __restrict__ qbar, const float* __restrict__ kbT,
+                                                     float* __restrict__ lg, int Tm, int Tn, int TnP,
+                                                     float inv_sqrt_d) {
+  __shared__ __align__(16) float qs[D * LG_ROWS];
+  pdl_wait();     // Qbar and Kbar^T are complete
+  pdl_trigger();  // the select kernel may be scheduled; it waits for this grid itself
+  const long long h = blockIdx.z;
+  const int i0 = blockIdx.y * LG_ROWS;
+  const int rc = min(LG_ROWS, Tm - i0);
+  for (int x = threadIdx.x; x < LG_ROWS * D; x += 256) {
+    const int r = x / D, dd = x % D;
+    qs[dd * LG_ROWS + r] = r < rc ? qbar[(h * Tm + i0 + r) * D + dd] : 0.f;
   }
   __syncthreads();
-  const WaitCtx wc{&abort_flag, status, wait_limit_ns};
-  int issued = 0;  // meaningful in thread 0 only
-  auto issue = [&](int ch) {  // thread 0 only
-    const int rows = min(KCH, Tn - ch * KCH);
-    const uint32_t bytes = (uint32_t)rows * D * 4;
-    uint64_t* bar = &full[ch % NST];
-    mbar_expect_tx(bar, bytes);
-    bulk_load(ring + (ch % NST) * KCH * D, kb + (long long)ch * KCH * D, bytes, bar);
-    issued = ch + 1;
-  };
-  if (threadIdx.x == 0)
-    for (int ch = 0; ch < min(NST - 1, nch); ++ch) issue(ch);
-  for (int e = threadIdx.x; e < ROWS * D; e += 256) {
-    const int rr = e / D;
-    qb[e] = (i0 + rr < Tm) ? qbar[(h * Tm + i0 + rr) * D + (e % D)] : 0.f;
-  }
-  __syncthreads();
-  float* lrow = lrows + warp * 32 * E;
-  const float4* qr = reinterpret_cast<const float4*>(qb + warp * D);
-  bool ok = true;
-  int ch = 0;
-  for (; ch < nch; ++ch) {
-    if (threadIdx.x == 0 && ch + NST - 1 < nch) issue(ch + NST - 1);  // its slot was freed last iteration
-    ok = wait_bar(&full[ch % NST], (ch / NST) & 1, wc);
-    if (__syncthreads_or(!ok)) {
-      ok = false;
-      break;
-    }
-    // lane l: logit of row (i0 + warp) against Kbar row ch*KCH + l; each lane walks
-    // d in its own rotated order (conflict-free 16-byte smem reads), sequentially
-    const int c = ch * KCH + (int)lane;
-    if (c < Tn) {
-      const float4* kr = reinterpret_cast<const float4*>(ring + (ch % NST) * KCH * D + lane * D);
-      float acc = 0.f;
-#pragma unroll 8
-      for (int t = 0; t < D / 4; ++t) {
-        const int e = (t + (int)lane) & (D / 4 - 1);
-        const float4 kv = kr[e];
-        const float4 qv = qr[e];
-        acc = fmaf(qv.x, kv.x, acc);
-        acc = fmaf(qv.y, kv.y, acc);
-        acc = fmaf(qv.z, kv.z, acc);
-        acc = fmaf(qv.w, kv.w, acc);
-      }
-      lrow[c] = acc * inv_sqrt_d;
-    }
-    __syncthreads();  // every warp is done with this slot
-  }
-  if (!ok) {
-    // never leave with bulk copies in flight: wait (bounded) for the issued ones
-    if (threadIdx.x == 0) {
-      __shared__ int never;
-      never = 0;
-      const WaitCtx dw{&never, nullptr, wait_limit_ns};
-      for (int c2 = ch; c2 < issued; ++c2) wait_bar(&full[c2 % NST], (c2 / NST) & 1, dw);
-    }
-    return;
-  }
-  const int i = i0 + warp;
-  if (i >= Tm) return;
-  float mx = -INFINITY;
-  for (int j = lane; j < Tn; j += 32) mx = fmaxf(mx, lrow[j]);
+  const int kp = (int)threadIdx.x & 63, hq = (int)threadIdx.x >> 6;
+  const int key = blockIdx.x * LG_KEYS + 2 * kp;
+  if (key >= Tn || hq * 4 >= rc) return;
+  float a0[4], a1[4];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffff, mx, o));
-  float ssum = 0.f;
-  for (int j = lane; j < Tn; j += 32) {
-    const float e = expf(lrow[j] - mx);
-    lrow[j] = e;
-    ssum += e;
+  for (int r = 0; r < 4; ++r) a0[r] = a1[r] = 0.f;
+  const float2* kcol = reinterpret_cast<const float2*>(kbT + h * D * TnP + key);
+#pragma unroll 16
+  for (int dd = 0; dd < D; ++dd) {
+    const float2 kv = __ldg(kcol + (long long)dd * (TnP / 2));
+    const float4 qq = *reinterpret_cast<const float4*>(qs + dd * LG_ROWS + hq * 4);
+    a0[0] = fmaf(kv.x, qq.x, a0[0]);
+    a1[0] = fmaf(kv.y, qq.x, a1[0]);
+    a0[1] = fmaf(kv.x, qq.y, a0[1]);
+    a1[1] = fmaf(kv.y, qq.y, a1[1]);
+    a0[2] = fmaf(kv.x, qq.z, a0[2]);
+    a1[2] = fmaf(kv.y, qq.z, a1[2]);
+    a0[3] = fmaf(kv.x, qq.w, a0[3]);
+    a1[3] = fmaf(kv.y, qq.w, a1[3]);
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ssum += __shfl_xor_sync(0xffffffff, ssum, o);
-  const long long rowid = h * Tm + i;
-  for (int j = lane; j < Tn; j += 32) {
-    const float p = lrow[j] / ssum;
-    lrow[j] = p;
-    if (out.pbar) out.pbar[rowid * Tn + j] = p;
+  for (int r = 0; r < 4; ++r) {
+    const int row = hq * 4 + r;
+    if (row < rc) {
+      float* dst = lg + (h * Tm + i0 + row) * Tn + key;
+      dst[0] = a0[r] * inv_sqrt_d;
+      if (key + 1 < Tn) dst[1] = a1[r] * inv_sqrt_d;
+    }
   }
-  __syncwarp();
-  select_row<E>(lrow, Tn, K, thr, out.row_cnt + rowid, out.row_idx + rowid * Tn, bits + rowid * W,
-                out.bitmap ? out.bitmap + rowid * Tn : nullptr, status);
+}
+
+// Softmax and selection, one warp per P-bar row (4 rows per CTA): the row's
+// logits from lg, P-bar in registers, CSR, kept-bit words, optional P-bar /
+// uint8 bitmap.
+template <int E>
+__global__ void __launch_bounds__(128, (E <= 16 ? 6 : 2)) select_kernel(const float* __restrict__ lg, long long R,
+                                                                       int Tn, int W, int K, unsigned long long thr,
+                                                                       MaskOut out, uint32_t* __restrict__ bits,
+                                                                       int* status) {
+  __shared__ uint32_t scr[4][96];
+  pdl_wait();     // the logits are complete
+  pdl_trigger();  // the CSC kernel may be scheduled; it waits for this grid itself
+  const int warp = (int)(threadIdx.x >> 5);
+  const long long rowid = (long long)blockIdx.x * 4 + warp;
+  if (rowid >= R) return;
+  softmax_select_row<E>(lg + rowid * Tn, Tn, K, thr, out.pbar ? out.pbar + rowid * Tn : nullptr, out.row_cnt + rowid,
+                        out.row_idx + rowid * Tn, bits + rowid * W, out.bitmap ? out.bitmap + rowid * Tn : nullptr,
+                        status, scr[warp]);
 }
 
 // selection alone on a given P-bar: one warp per row, 8 rows per CTA
@@ -358,74 +569,83 @@ template <int E>
 __global__ void __launch_bounds__(256) pbar_select_kernel(const float* __restrict__ pbar, int Tm, int Tn, int W,
                                                           int K, unsigned long long thr, MaskOut out,
                                                           uint32_t* __restrict__ bits, int* status) {
+  pdl_trigger();
   const int w = threadIdx.x >> 5;
   const long long bh = blockIdx.y;
   const int i = blockIdx.x * 8 + w;
   if (i >= Tm) return;
+  __shared__ uint32_t scr[8][96];
   const long long rowid = bh * Tm + i;
   select_row<E>(pbar + rowid * Tn, Tn, K, thr, out.row_cnt + rowid, out.row_idx + rowid * Tn, bits + rowid * W,
-                out.bitmap ? out.bitmap + rowid * Tn : nullptr, status);
+                out.bitmap ? out.bitmap + rowid * Tn : nullptr, status, scr[w]);
 }
 
-// kept-bit words [B*H, Tm, W] -> CSC; one warp per kv-block column, 8 per CTA
-__global__ void __launch_bounds__(256) csc_kernel(const uint32_t* __restrict__ bits, int h0, int Tm, int Tn,
-                                                  int W, int* __restrict__ col_cnt, int* __restrict__ col_idx) {
-  const long long bh = h0 + blockIdx.y;
-  const int c = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (c >= Tn) return;
-  csc_column_warp(bits + bh * Tm * W, Tm, W, c, col_cnt + bh * Tn + c, col_idx + (bh * Tn + c) * Tm);
+// kept-bit words [B*H, Tm, W] -> CSC; one CTA per (32-column word, head)
+__global__ void __launch_bounds__(256) csc_kernel(const uint32_t* __restrict__ bits, int Tm, int Tn, int W,
+                                                  int* __restrict__ col_cnt, int* __restrict__ col_idx) {
+  __shared__ int cnt_smem[8 * 32];
+  __shared__ int base_smem[32];
+  pdl_wait();  // the kept-bit words are complete
+  const long long bh = blockIdx.y;
+  csc_word_cta(bits + bh * Tm * W, Tm, Tn, W, blockIdx.x, col_cnt + bh * Tn, col_idx + bh * Tn * Tm, cnt_smem,
+               base_smem);
 }
 
 // ---------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------
-template <int D, int E>
-static cudaError_t launch_select_t(const float* qbar, const float* kbar, int h0, int nh, int Tm, int Tn, int W, int K,
-                                   unsigned long long thr, const MaskOut& out, uint32_t* bits, int* status,
-                                   unsigned long long wait_limit_ns, cudaStream_t s) {
-  const size_t smem = ((size_t)4 * KCH * D + (size_t)ROWS * D + (size_t)ROWS * 32 * E) * 4 + 4 * 8;
-  cudaError_t e = cudaFuncSetAttribute(select_kernel<D, E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
+int kbar_cols(int Tn) { return (Tn + 3) & ~3; }
+
+template <int E>
+static cudaError_t launch_select_t(const float* lg, int BH, int Tm, int Tn, int W, int K, unsigned long long thr,
+                                   const MaskOut& out, uint32_t* bits, int* status, cudaStream_t s) {
+  const long long R = (long long)BH * Tm;
   KernelTimer kt(KID_SELECT, s);
-  select_kernel<D, E><<<dim3((Tm + ROWS - 1) / ROWS, nh), 256, smem, s>>>(
-      qbar, kbar, h0, Tm, Tn, W, 1.0f / sqrtf((float)D), K, thr, out, bits, status, wait_limit_ns);
-  return cudaGetLastError();
+  return launch_k(select_kernel<E>, dim3((unsigned)((R + 3) / 4)), dim3(128), 0, s, true, lg, R, Tn, W, K, thr, out,
+                  bits, status);
+}
+
+static cudaError_t launch_select_e(const float* lg, int BH, int Tm, int Tn, int W, int K, unsigned long long thr,
+                                   const MaskOut& out, uint32_t* bits, int* status, cudaStream_t s) {
+  const int e = (Tn + 31) / 32;
+  if (e <= 8) return launch_select_t<8>(lg, BH, Tm, Tn, W, K, thr, out, bits, status, s);
+  if (e <= 16) return launch_select_t<16>(lg, BH, Tm, Tn, W, K, thr, out, bits, status, s);
+  if (e <= 40) return launch_select_t<40>(lg, BH, Tm, Tn, W, K, thr, out, bits, status, s);
+  return launch_select_t<64>(lg, BH, Tm, Tn, W, K, thr, out, bits, status, s);
 }
 
 template <int D>
-static cudaError_t launch_select_d(const float* qbar, const float* kbar, int h0, int nh, int Tm, int Tn, int W, int K,
-                                   unsigned long long thr, const MaskOut& out, uint32_t* bits, int* status,
-                                   unsigned long long wl, cudaStream_t s) {
-  const int e = (Tn + 31) / 32;
-  if (e <= 8) return launch_select_t<D, 8>(qbar, kbar, h0, nh, Tm, Tn, W, K, thr, out, bits, status, wl, s);
-  if (e <= 16) return launch_select_t<D, 16>(qbar, kbar, h0, nh, Tm, Tn, W, K, thr, out, bits, status, wl, s);
-  if (e <= 40) return launch_select_t<D, 40>(qbar, kbar, h0, nh, Tm, Tn, W, K, thr, out, bits, status, wl, s);
-  return launch_select_t<D, 64>(qbar, kbar, h0, nh, Tm, Tn, W, K, thr, out, bits, status, wl, s);
+static cudaError_t launch_logits_d(const float* qbar, const float* kbT, float* lg, int BH, int Tm, int Tn,
+                                   cudaStream_t s) {
+  KernelTimer kt(KID_LOGITS, s);
+  return launch_k(logits_kernel<D>, dim3((Tn + LG_KEYS - 1) / LG_KEYS, (Tm + LG_ROWS - 1) / LG_ROWS, BH), dim3(256),
+                  0, s, true, qbar, kbT, lg, Tm, Tn, kbar_cols(Tn), 1.0f / sqrtf((float)D));
 }
 
-cudaError_t launch_mask(const void* q, const void* k, float* qbar, float* kbar, int BH, int N, int d, int Tm, int Tn,
-                        int bq, int bkv, int K, unsigned long long thr, const MaskOut& out, int* col_cnt,
-                        int* col_idx, uint32_t* bits, int W, int* status, unsigned long long wait_limit_ns,
-                        cudaStream_t s) {
-  dim3 grid(Tm + Tn, BH);
-  {
+template <int D>
+static cudaError_t launch_pool_d(const void* q, const void* k, float* qbar, float* kbT, int BH, int N, int Tm, int Tn,
+                                 int bq, int bkv, cudaStream_t s) {
   KernelTimer kt(KID_POOL, s);
-  if (d == 128)
-    pool_kernel<128><<<grid, 256, 0, s>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qbar, kbar, 0, N, Tm, Tn,
-                                          bq, bkv);
-  else
-    pool_kernel<64><<<grid, 256, 0, s>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, qbar, kbar, 0, N, Tm, Tn,
-                                         bq, bkv);
-  }
-  cudaError_t e = cudaGetLastError();
+  return launch_k(pool_kernel<D>, dim3(Tm + Tn, BH), dim3(256), 0, s, false, static_cast<const __nv_bfloat16*>(q),
+                  static_cast<const __nv_bfloat16*>(k), qbar, kbT, N, Tm, Tn, kbar_cols(Tn), bq, bkv);
+}
+
+cudaError_t launch_mask(const void* q, const void* k, float* qbar, float* kbT, float* lg, int BH, int N, int d,
+                        int Tm, int Tn, int bq, int bkv, int K, unsigned long long thr, const MaskOut& out,
+                        int* col_cnt, int* col_idx, uint32_t* bits, int W, int* status,
+                        unsigned long long wait_limit_ns, cudaStream_t s) {
+  (void)wait_limit_ns;
+  cudaError_t e = d == 128 ? launch_pool_d<128>(q, k, qbar, kbT, BH, N, Tm, Tn, bq, bkv, s)
+                           : launch_pool_d<64>(q, k, qbar, kbT, BH, N, Tm, Tn, bq, bkv, s);
   if (e != cudaSuccess) return e;
-  e = (d == 128) ? launch_select_d<128>(qbar, kbar, 0, BH, Tm, Tn, W, K, thr, out, bits, status, wait_limit_ns, s)
-                 : launch_select_d<64>(qbar, kbar, 0, BH, Tm, Tn, W, K, thr, out, bits, status, wait_limit_ns, s);
+  e = d == 128 ? launch_logits_d<128>(qbar, kbT, lg, BH, Tm, Tn, s) : launch_logits_d<64>(qbar, kbT, lg, BH, Tm, Tn, s);
+  if (e != cudaSuccess) return e;
+  e = launch_select_e(lg, BH, Tm, Tn, W, K, thr, out, bits, status, s);
   if (e != cudaSuccess) return e;
   if (col_cnt) {
     KernelTimer kt(KID_CSC, s);
-    csc_kernel<<<dim3((Tn + 7) / 8, BH), 256, 0, s>>>(bits, 0, Tm, Tn, W, col_cnt, col_idx);
-    e = cudaGetLastError();
+    e = launch_k(csc_kernel, dim3(W, BH), dim3(256), 0, s, true, static_cast<const uint32_t*>(bits), Tm, Tn, W,
+                 col_cnt, col_idx);
   }
   return e;
 }
@@ -448,10 +668,8 @@ cudaError_t launch_select(const float* pbar, int BH, int Tm, int Tn, int K, unsi
 
 cudaError_t launch_csc(const uint32_t* bits, int BH, int Tm, int Tn, int W, int* col_cnt, int* col_idx,
                        cudaStream_t s) {
-  dim3 grid((Tn + 7) / 8, BH);
   KernelTimer kt(KID_CSC, s);
-  csc_kernel<<<grid, 256, 0, s>>>(bits, 0, Tm, Tn, W, col_cnt, col_idx);
-  return cudaGetLastError();
+  return launch_k(csc_kernel, dim3(W, BH), dim3(256), 0, s, true, bits, Tm, Tn, W, col_cnt, col_idx);
 }
 
 }  // namespace spa2

@@ -16,6 +16,7 @@ namespace {
 const char* const kNames[KID_COUNT] = {
     "pool_kernel",        // KID_POOL
     "select_kernel",      // KID_SELECT
+    "logits_kernel",      // KID_LOGITS
     "csc_kernel",         // KID_CSC
     "pbar_select_kernel", // KID_PBAR_SELECT
     "v_to_f16_kernel",    // KID_V16
