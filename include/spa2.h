@@ -19,8 +19,13 @@
  *   device memory, 16-byte aligned. LSE is [B, H, N] fp32 (natural log of the
  *   row sum of exp(scaled logits)). Block counts: T_m = ceil(N / bq),
  *   T_n = ceil(N / bkv); the last block of a ragged N is partial.
- * Supported set. d in {64, 128}; (bq, bkv) = (128, 64); N >= 1; B, H >= 1;
- *   0 <= k_frac <= 1, 0 <= p_frac <= 1. Anything else returns
+ * Supported set. d in {64, 128}; bq in {64, 128, 256}; bkv in {64, 128};
+ *   1 <= N <= 131072; B, H >= 1 with B*H <= 65535; 0 <= k_frac <= 1,
+ *   0 <= p_frac <= 1. (bq, bkv) = (128, 64) is the method's setting and the
+ *   fastest path; the other sizes run the same attention kernels on tiles of
+ *   128 query rows x 64 key rows through tile lists built at the start of the
+ *   forward / backward call (per-layer block sizes: paper.rainbus.top,
+ *   独立分析的弱点). Anything else returns
  *   SPA2_ERR_UNSUPPORTED (or SPA2_ERR_INVALID_ARG for nonsense such as a null
  *   pointer or a negative size) and launches nothing.
  * Ownership. The caller allocates and owns every buffer, including the
@@ -190,7 +195,8 @@ SPA2_API spa2_status spa2_select_blocks(const float* pbar, int B, int H, int Tm,
  *                   bits); pass it to the backward for an accurate
  *                   D = rowsum(dO * O). NULL skips it.
  *   lse           : [B, H, N] fp32 device output (natural-log LSE)
- *   ws            : spa2_workspace_bytes(SPA2_OP_FWD, ...) bytes
+ *   ws            : spa2_workspace_bytes(SPA2_OP_FWD, ...) bytes (fp16 copy of
+ *                   V, and the tile lists for sizes other than (128, 64))
  */
 SPA2_API spa2_status spa2_sparse_attn_fwd(const void* q, const void* k, const void* v, int B, int H, int N, int d,
                                           int bq, int bkv, const spa2_mask* mask, float softmax_scale, void* o,
@@ -223,8 +229,9 @@ SPA2_API spa2_status spa2_sparse_attn_fwd(const void* q, const void* k, const vo
  *                      col_cnt/col_idx are read
  *   dq, dk, dv       : [B, H, N, d] device outputs of type grad_dtype
  *   grad_dtype       : SPA2_DTYPE_BF16 or SPA2_DTYPE_F32
- *   ws               : spa2_workspace_bytes(SPA2_OP_BWD, ...) bytes (holds D
- *                      and the fp16 copies of dO, V, Q and K)
+ *   ws               : spa2_workspace_bytes(SPA2_OP_BWD, ...) bytes (holds D,
+ *                      the fp16 copies of dO, V, Q and K, and the tile lists
+ *                      for sizes other than (128, 64))
  */
 SPA2_API spa2_status spa2_sparse_attn_bwd(const void* q, const void* k, const void* v, const void* o,
                                           const void* o_lo, const float* lse, const void* dout, int B, int H, int N,

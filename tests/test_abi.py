@@ -46,7 +46,13 @@ def test_workspace_sizes(L):
     assert b.spa2_workspace_bytes(b.OP_SELECT, 2, 3, 5, 40, 0, 0) == 256 + 256   # 2*3*5*2 words = 240 B
     # unsupported shapes report 0
     assert b.spa2_workspace_bytes(b.OP_MASK, 1, 1, 100, 96) == 0
-    assert b.spa2_workspace_bytes(b.OP_MASK, 1, 1, 100, 128, 64, 64) == 0
+    assert b.spa2_workspace_bytes(b.OP_MASK, 1, 1, 100, 128, 32, 64) == 0
+    assert b.spa2_workspace_bytes(b.OP_MASK, 1, 1, 100, 128, 128, 256) == 0
+    for bq in (64, 128, 256):
+        for bkv in (64, 128):
+            assert b.spa2_workspace_bytes(b.OP_FWD, 1, 2, 1000, 128, bq, bkv) > 0
+    # tile lists are extra workspace only for sizes other than (128, 64)
+    assert b.spa2_workspace_bytes(b.OP_FWD, 1, 2, 1000, 128, 64, 128) > b.spa2_workspace_bytes(b.OP_FWD, 1, 2, 1000, 128)
     assert b.spa2_workspace_bytes(b.OP_MASK, 1, 1, 0, 128) == 0
 
 
@@ -58,7 +64,7 @@ def test_argument_errors_are_synchronous(L):
     m = b.spa2_mask(fake, fake, None, None, None, None)
     # unsupported head dim / block sizes / fractions
     assert b.spa2_block_mask(fake, fake, 1, 1, 128, 96, 128, 64, 0.1, 0.5, m, fake, 1 << 30, None) == b.ERR_UNSUPPORTED
-    assert b.spa2_block_mask(fake, fake, 1, 1, 128, 128, 64, 64, 0.1, 0.5, m, fake, 1 << 30, None) == b.ERR_UNSUPPORTED
+    assert b.spa2_block_mask(fake, fake, 1, 1, 128, 128, 96, 64, 0.1, 0.5, m, fake, 1 << 30, None) == b.ERR_UNSUPPORTED
     assert b.spa2_block_mask(fake, fake, 1, 1, 128, 128, 128, 64, 1.5, 0.5, m, fake, 1 << 30, None) == b.ERR_UNSUPPORTED
     assert b.spa2_block_mask(fake, fake, 1, 1, 128, 128, 128, 64, float("nan"), 0.5, m, fake, 1 << 30,
                              None) == b.ERR_UNSUPPORTED

@@ -292,3 +292,68 @@ def test_wan14b_fwd_bwd_sampled():
                 acc["dV"].add(dv[0, hi, j * 64:j * 64 + gv.shape[0]], gv)
     for a in acc.values():
         a.check()
+
+
+@pytest.mark.parametrize("bq,bkv", [(64, 64), (64, 128), (128, 128), (256, 64), (256, 128)])
+@pytest.mark.parametrize("N,d", [(1000, 128), (777, 64)])
+def test_block_sizes_mask_fwd_bwd(bq, bkv, N, d):
+    """Block sizes other than (128, 64) (per-layer block sizes): pooled softmax and
+    selection (bit-exact on the GPU's own P-bar) with the oracle's block
+    partition, CSC, then O, LSE, dQ, dK, dV against the oracle under that mask.
+    N = 1000 and 777 leave ragged last blocks of every size (777 with b_q = 64
+    leaves the last 128-row query tile half empty)."""
+    from tests._parity import csc_to_dense
+    B, H = 1, 2
+    q, k, v = synth.gaussian_with_sinks(B=B, H=H, N=N, d=d, seed=bq * 7 + bkv + N, device="cuda")
+    dout = synth.normal_like(q.shape, seed=N + bq + bkv, device="cuda")
+    s = b.Spa2(B, H, N, d, bq=bq, bkv=bkv, with_pbar=True)
+    kf, pf = 0.15, 0.5
+    m = s.block_mask(q, k, kf, pf)
+    o, lse = s.fwd(q, k, v, m)
+    grads = s.bwd(q, k, v, o, lse, dout, m)
+    s.check()
+    Tm, Tn = oracle.block_counts(N, bq, bkv)
+    assert (s.Tm, s.Tn) == (Tm, Tn)
+    pbar = m.pbar.cpu().numpy()
+    pbar64 = oracle.pooled_attention(oracle.pool_blocks(f64(q), bq), oracle.pool_blocks(f64(k), bkv), d)
+    np.testing.assert_allclose(pbar, pbar64, rtol=0, atol=1e-5)
+    dense = csr_to_dense(m.row_cnt.cpu().numpy(), m.row_idx.cpu().numpy(), Tn)
+    np.testing.assert_array_equal(dense, oracle.select_blocks(pbar, kf, pf))
+    np.testing.assert_array_equal(csc_to_dense(m.col_cnt.cpu().numpy(), m.col_idx.cpu().numpy(), Tm), dense)
+    O, LSE = oracle.masked_attn_fwd(f64(q), f64(k), f64(v), dense, bq, bkv)
+    assert_close(_o32(s, o), O, "O (o + o_lo)")
+    assert_close_bf16_out(f64(o), O, "O (bf16)")
+    assert_close(lse.cpu().numpy(), LSE, "LSE")
+    dQ, dK, dV = oracle.masked_attn_bwd(f64(q), f64(k), f64(v), dense, f64(dout), bq, bkv)
+    assert_close(f64(grads[0]), dQ, "dQ")
+    assert_close(f64(grads[1]), dK, "dK")
+    assert_close(f64(grads[2]), dV, "dV")
+
+
+def test_block_size_64_rows_with_disjoint_halves():
+    """b_q = 64 where the two query blocks sharing a 128-row tile keep disjoint
+    kv-blocks (from a hand-made P-bar): every tile entry excludes one half, and
+    the rows of each half must see only their own block's keys."""
+    B, H, N, d = 1, 1, 512, 128
+    q, k, v = synth.gaussian_with_sinks(B=B, H=H, N=N, d=d, seed=77, device="cuda")
+    dout = synth.normal_like(q.shape, seed=78, device="cuda")
+    Tm, Tn = oracle.block_counts(N, 64, 64)                      # 8 x 8
+    pbar = np.full((B, H, Tm, Tn), 1e-4, dtype=np.float32)
+    for i in range(Tm):                                          # even blocks keep kv 0..3, odd ones 4..7
+        cols = range(0, 4) if i % 2 == 0 else range(4, 8)
+        for j in cols:
+            pbar[0, 0, i, j] = 0.2
+    mask = b.select_blocks(torch.tensor(pbar, device="cuda"), 0.5, 0.0)
+    s = b.Spa2(B, H, N, d, bq=64, bkv=64)
+    o, lse = s.fwd(q, k, v, mask)
+    grads = s.bwd(q, k, v, o, lse, dout, mask)
+    s.check()
+    dense = csr_to_dense(mask.row_cnt.cpu().numpy(), mask.row_idx.cpu().numpy(), Tn)
+    assert dense[0, 0, 0, :4].all() and not dense[0, 0, 0, 4:].any() and dense[0, 0, 1, 4:].all()
+    O, LSE = oracle.masked_attn_fwd(f64(q), f64(k), f64(v), dense, 64, 64)
+    assert_close(_o32(s, o), O, "O (o + o_lo)")
+    assert_close(lse.cpu().numpy(), LSE, "LSE")
+    dQ, dK, dV = oracle.masked_attn_bwd(f64(q), f64(k), f64(v), dense, f64(dout), 64, 64)
+    assert_close(f64(grads[0]), dQ, "dQ")
+    assert_close(f64(grads[1]), dK, "dK")
+    assert_close(f64(grads[2]), dV, "dV")

@@ -78,12 +78,12 @@ class _StatusWatch:
                 raise b.Spa2Error(code, f"device status of sparse_attention (op {op})")
 
 
-def _spa(B, H, N, d, device) -> b.Spa2:
+def _spa(B, H, N, d, device, bq=b.BQ, bkv=b.BKV) -> b.Spa2:
     stream = torch.cuda.current_stream(device).cuda_stream
-    key = (B, H, N, d, str(device), stream)
+    key = (B, H, N, d, bq, bkv, str(device), stream)
     s = _cache.get(key)
     if s is None:
-        s = _cache[key] = b.Spa2(B, H, N, d, device=device)
+        s = _cache[key] = b.Spa2(B, H, N, d, device=device, bq=bq, bkv=bkv)
         s.watch = _StatusWatch(s)
     s.watch.poll()
     return s
@@ -106,12 +106,13 @@ class SparseAttentionFunction(torch.autograd.Function):
     """
 
     @staticmethod
-    def forward(ctx, q, k, v, k_frac: float, p_frac: float, scale: float = 0.0, mask: b.Mask | None = None):
+    def forward(ctx, q, k, v, k_frac: float, p_frac: float, scale: float = 0.0, mask: b.Mask | None = None,
+                bq: int = b.BQ, bkv: int = b.BKV):
         if q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16 or v.dtype != torch.bfloat16:
             raise TypeError("sparse_attention expects bf16 q, k, v")
         q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
         B, H, N, d = q.shape
-        s = _spa(B, H, N, d, q.device)
+        s = _spa(B, H, N, d, q.device, bq, bkv)
         ops = [b.OP_FWD]
         if mask is None:
             mask = s.block_mask(q, k, k_frac, p_frac)
@@ -134,28 +135,29 @@ class SparseAttentionFunction(torch.autograd.Function):
         dq, dk, dv = ctx.spa.bwd(q, k, v, o, lse, do.contiguous(), ctx.mask, ctx.scale, o_lo=o_lo,
                                  grad_dtype=b.DTYPE_BF16)
         ctx.spa.watch.after([b.OP_BWD])
-        return dq, dk, dv, None, None, None, None
+        return dq, dk, dv, None, None, None, None, None, None
 
 
-def block_mask(q, k, k_frac: float, p_frac: float) -> b.Mask:
+def block_mask(q, k, k_frac: float, p_frac: float, bq: int = b.BQ, bkv: int = b.BKV) -> b.Mask:
     """The hybrid block mask of (q, k) alone (CSR and CSC on the device), for
     reuse through `sparse_attention(..., mask=...)`."""
     if q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16:
         raise TypeError("block_mask expects bf16 q, k")
     q, k = q.contiguous(), k.contiguous()
     B, H, N, d = q.shape
-    s = _spa(B, H, N, d, q.device)
+    s = _spa(B, H, N, d, q.device, bq, bkv)
     m = s.block_mask(q, k, k_frac, p_frac)
     s.watch.after([b.OP_MASK])
     return m
 
 
 def sparse_attention(q, k, v, k_frac: float = 0.0, p_frac: float = 0.0, scale: float = 0.0,
-                     return_mask: bool = False, mask: b.Mask | None = None):
-    """Differentiable hybrid block-sparse attention (b_q = 128, b_kv = 64).
+                     return_mask: bool = False, mask: b.Mask | None = None, bq: int = b.BQ, bkv: int = b.BKV):
+    """Differentiable hybrid block-sparse attention with query blocks of bq rows
+    (64, 128 or 256) and key/value blocks of bkv rows (64 or 128).
 
-    With `mask` (from `block_mask` on a problem of the same shape) the given
-    mask is used as is and k_frac, p_frac are ignored.
+    With `mask` (from `block_mask` on a problem of the same shape and block
+    sizes) the given mask is used as is and k_frac, p_frac are ignored.
     """
-    o, row_cnt = SparseAttentionFunction.apply(q, k, v, k_frac, p_frac, scale, mask)
+    o, row_cnt = SparseAttentionFunction.apply(q, k, v, k_frac, p_frac, scale, mask, bq, bkv)
     return (o, row_cnt) if return_mask else o

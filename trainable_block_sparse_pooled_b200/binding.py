@@ -196,8 +196,8 @@ class Mask:
         return int(self.row_cnt.sum().item())
 
 
-def block_counts(N: int) -> tuple[int, int]:
-    return math.ceil(N / BQ), math.ceil(N / BKV)
+def block_counts(N: int, bq: int = BQ, bkv: int = BKV) -> tuple[int, int]:
+    return math.ceil(N / bq), math.ceil(N / bkv)
 
 
 def _stream(torch):
@@ -211,16 +211,17 @@ class Spa2:
     caller side of the ABI; the library itself never allocates.
     """
 
-    def __init__(self, B, H, N, d, device="cuda", with_pbar=False, with_bitmap=False):
+    def __init__(self, B, H, N, d, device="cuda", with_pbar=False, with_bitmap=False, bq=BQ, bkv=BKV):
         import torch
         self.torch = torch
         self.B, self.H, self.N, self.d = B, H, N, d
-        self.Tm, self.Tn = block_counts(N)
+        self.bq, self.bkv = bq, bkv
+        self.Tm, self.Tn = block_counts(N, bq, bkv)
         self.device = device
         L = lib()
-        self.ws_bytes = {op: L.spa2_workspace_bytes(op, B, H, N, d, BQ, BKV) for op in (OP_MASK, OP_FWD, OP_BWD)}
+        self.ws_bytes = {op: L.spa2_workspace_bytes(op, B, H, N, d, bq, bkv) for op in (OP_MASK, OP_FWD, OP_BWD)}
         if min(self.ws_bytes.values()) == 0:
-            raise Spa2Error(ERR_UNSUPPORTED, f"shape B={B} H={H} N={N} d={d}")
+            raise Spa2Error(ERR_UNSUPPORTED, f"shape B={B} H={H} N={N} d={d} bq={bq} bkv={bkv}")
         # zero-filled so that the status word of an op never run reads as OK
         self.ws = {op: torch.zeros(n, dtype=torch.uint8, device=device) for op, n in self.ws_bytes.items()}
         self.with_pbar, self.with_bitmap = with_pbar, with_bitmap
@@ -237,7 +238,8 @@ class Spa2:
         mask = mask or self.new_mask()
         cm = mask.c()
         ws = self.ws[OP_MASK]
-        _check(spa2_block_mask(q.data_ptr(), k.data_ptr(), self.B, self.H, self.N, self.d, BQ, BKV, float(k_frac),
+        _check(spa2_block_mask(q.data_ptr(), k.data_ptr(), self.B, self.H, self.N, self.d, self.bq, self.bkv,
+                               float(k_frac),
                                float(p_frac), cm, ws.data_ptr(), ws.numel(), _stream(self.torch)), "spa2_block_mask")
         return mask
 
@@ -250,8 +252,8 @@ class Spa2:
         lse = t.empty(self.B, self.H, self.N, dtype=t.float32, device=q.device) if lse is None else lse
         cm = mask.c()
         ws = self.ws[OP_FWD]
-        _check(spa2_sparse_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), self.B, self.H, self.N, self.d, BQ,
-                                    BKV, cm, float(scale), o.data_ptr(), None if o_lo is None else o_lo.data_ptr(),
+        _check(spa2_sparse_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), self.B, self.H, self.N, self.d, self.bq,
+                                    self.bkv, cm, float(scale), o.data_ptr(), None if o_lo is None else o_lo.data_ptr(),
                                     lse.data_ptr(), ws.data_ptr(), ws.numel(), _stream(t)), "spa2_sparse_attn_fwd")
         self.o_lo = o_lo
         return o, lse
@@ -270,7 +272,7 @@ class Spa2:
         ws = self.ws[OP_BWD]
         _check(spa2_sparse_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                                     None if o_lo is None else o_lo.data_ptr(), lse.data_ptr(), dout.data_ptr(),
-                                    self.B, self.H, self.N, self.d, BQ, BKV, cm, float(scale), dq.data_ptr(),
+                                    self.B, self.H, self.N, self.d, self.bq, self.bkv, cm, float(scale), dq.data_ptr(),
                                     dk.data_ptr(), dv.data_ptr(), int(grad_dtype), ws.data_ptr(), ws.numel(),
                                     _stream(t)), "spa2_sparse_attn_bwd")
         return dq, dk, dv

@@ -18,7 +18,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libspa2.so")
-SOURCES = ["api.cu", "mask.cu", "attn_fwd.cu", "attn_bwd.cu", "noalloc.cu", "timing.cu"]
+SOURCES = ["api.cu", "mask.cu", "attn_fwd.cu", "attn_bwd.cu", "noalloc.cu", "timing.cu", "tiles.cu"]
 HEADERS = ["common.cuh", "kernels.h"]
 
 NVCC_FLAGS = [

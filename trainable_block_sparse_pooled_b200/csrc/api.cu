@@ -20,6 +20,9 @@ static inline size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
 struct Shape {
   int B, H, N, d, Tm, Tn, W;
   long long BH;
+  int bq, bkv;
+  int TMt, TNt;  // 128-row query tiles and 64-row key tiles of the attention kernels
+  bool tiled;    // block sizes other than (128, 64): the block lists are converted to tile lists
 };
 
 static bool shape_ok(int B, int H, int N, int d, int bq, int bkv, Shape* s, spa2_status* err) {
@@ -27,7 +30,8 @@ static bool shape_ok(int B, int H, int N, int d, int bq, int bkv, Shape* s, spa2
     *err = SPA2_ERR_INVALID_ARG;
     return false;
   }
-  if ((d != 64 && d != 128) || bq != 128 || bkv != 64 || N > 131072 || (long long)B * H > 65535) {
+  if ((d != 64 && d != 128) || (bq != 64 && bq != 128 && bq != 256) || (bkv != 64 && bkv != 128) || N > 131072 ||
+      (long long)B * H > 65535) {
     *err = SPA2_ERR_UNSUPPORTED;
     return false;
   }
@@ -39,6 +43,11 @@ static bool shape_ok(int B, int H, int N, int d, int bq, int bkv, Shape* s, spa2
   s->Tm = (N + bq - 1) / bq;
   s->Tn = (N + bkv - 1) / bkv;
   s->W = (s->Tn + 31) / 32;
+  s->bq = bq;
+  s->bkv = bkv;
+  s->TMt = (N + 127) / 128;
+  s->TNt = (N + 63) / 64;
+  s->tiled = bq != 128 || bkv != 64;
   return true;
 }
 
@@ -72,6 +81,46 @@ static MaskWs mask_ws(void* ws, const Shape& s) {
   return w;
 }
 
+// tile lists (tiled shapes only): CSR [BH, TMt] counts + [BH, TMt, TNt] entries,
+// CSC [BH, TNt] counts + [BH, TNt, TMt] entries
+struct TileWs {
+  int* csr_cnt;
+  int* csr_idx;
+  int* csc_cnt;
+  int* csc_idx;
+};
+static size_t tile_ws(char* base, size_t off, const Shape& s, bool csc, TileWs* t) {
+  if (!s.tiled) return off;
+  t->csr_cnt = reinterpret_cast<int*>(base + off);
+  off += al256((size_t)s.BH * s.TMt * 4);
+  t->csr_idx = reinterpret_cast<int*>(base + off);
+  off += al256((size_t)s.BH * s.TMt * s.TNt * 4);
+  if (csc) {
+    t->csc_cnt = reinterpret_cast<int*>(base + off);
+    off += al256((size_t)s.BH * s.TNt * 4);
+    t->csc_idx = reinterpret_cast<int*>(base + off);
+    off += al256((size_t)s.BH * s.TNt * s.TMt * 4);
+  }
+  return off;
+}
+
+struct FwdWs {
+  int* status;
+  void* v16;
+  TileWs tiles;
+  size_t bytes;
+};
+static FwdWs fwd_ws(void* ws, const Shape& s) {
+  FwdWs w{};
+  char* base = static_cast<char*>(ws);
+  size_t off = 256;
+  w.status = reinterpret_cast<int*>(base);
+  w.v16 = base + off;
+  off += al256((size_t)s.BH * s.N * s.d * 2);
+  w.bytes = tile_ws(base, off, s, false, &w.tiles);
+  return w;
+}
+
 struct BwdWs {
   int* status;
   float* dvec;
@@ -79,6 +128,7 @@ struct BwdWs {
   void* v16;
   void* q16;
   void* k16;
+  TileWs tiles;
   size_t bytes;
 };
 static BwdWs bwd_ws(void* ws, const Shape& s) {
@@ -96,7 +146,7 @@ static BwdWs bwd_ws(void* ws, const Shape& s) {
   off += al256((size_t)s.BH * s.N * s.d * 2);
   w.k16 = base + off;
   off += al256((size_t)s.BH * s.N * s.d * 2);
-  w.bytes = off;
+  w.bytes = tile_ws(base, off, s, true, &w.tiles);
   return w;
 }
 
@@ -251,7 +301,7 @@ size_t spa2_workspace_bytes(int op, int B, int H, int N, int d, int bq, int bkv)
   if (!shape_ok(B, H, N, d, bq, bkv, &s, &err)) return 0;
   switch (op) {
     case SPA2_OP_MASK: return mask_ws(nullptr, s).bytes;
-    case SPA2_OP_FWD: return 256 + al256((size_t)s.BH * s.N * s.d * 2);  // status + fp16 V
+    case SPA2_OP_FWD: return fwd_ws(nullptr, s).bytes;  // status + fp16 V (+ tile lists)
     case SPA2_OP_BWD: return bwd_ws(nullptr, s).bytes;
   }
   return 0;
@@ -314,19 +364,29 @@ spa2_status spa2_sparse_attn_fwd(const void* q, const void* k, const void* v, in
   if (!shape_ok(B, H, N, d, bq, bkv, &s, &err)) return err;
   if (!(softmax_scale >= 0.f) || isinf(softmax_scale)) return SPA2_ERR_UNSUPPORTED;
   if (!ws || !aligned(ws, 256)) return SPA2_ERR_WORKSPACE;
-  if (ws_bytes < 256 + al256((size_t)s.BH * s.N * s.d * 2)) return SPA2_ERR_WORKSPACE;
+  FwdWs w = fwd_ws(ws, s);
+  if (ws_bytes < w.bytes) return SPA2_ERR_WORKSPACE;
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)d);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  void* v16 = static_cast<char*>(ws) + 256;
+  void* v16 = w.v16;
   CUtensorMap tq, tk, tv, to, tolo;
   if (!make_map(&tq, q, s, 128) || !make_map(&tk, k, s, 64) || !make_map(&tv, v16, s, 64, true) ||
       !make_map(&to, o, s, 128) || !make_map(&tolo, o_lo ? o_lo : o, s, 128))
     return SPA2_ERR_CUDA;
-  int* status = static_cast<int*>(ws);
+  int* status = w.status;
   SPA2_CUDA_TRY(cudaMemsetAsync(status, 0, 4, st));
+  const int* rc = mask->row_cnt;
+  const int* ri = mask->row_idx;
+  if (s.tiled) {
+    SPA2_CUDA_TRY(launch_tile_lists(mask->row_cnt, mask->row_idx, nullptr, nullptr, (int)s.BH, s.Tm, s.Tn, s.TMt,
+                                    s.TNt, s.bq, s.bkv, w.tiles.csr_cnt, w.tiles.csr_idx, nullptr, nullptr, status,
+                                    st));
+    rc = w.tiles.csr_cnt;
+    ri = w.tiles.csr_idx;
+  }
   SPA2_CUDA_TRY(launch_v_to_f16(v, v16, s.BH * s.N * s.d, status, st));
-  FwdArgs a{&tq, &tk, &tv, &to, &tolo, o_lo != nullptr, mask->row_cnt, mask->row_idx, lse, (int)s.BH, s.N, s.Tm,
-            s.Tn, scale * 1.4426950408889634f, status, g_wait_limit_ns};
+  FwdArgs a{&tq, &tk, &tv, &to, &tolo, o_lo != nullptr, rc, ri, lse, (int)s.BH, s.N, s.TMt, s.TNt,
+            scale * 1.4426950408889634f, status, g_wait_limit_ns};
   SPA2_CUDA_TRY(launch_fwd(a, d, st));
   return SPA2_OK;
 }
@@ -358,8 +418,18 @@ spa2_status spa2_sparse_attn_bwd(const void* q, const void* k, const void* v, co
       !make_map(&tk16, w.k16, s, 64, true) || !(f32 ? make_map_f32(&tdq, dq, s, 128) : make_map(&tdq, dq, s, 128)))
     return SPA2_ERR_CUDA;
   SPA2_CUDA_TRY(cudaMemsetAsync(w.status, 0, 4, st));
-  BwdArgs a{&tq, &tk, &tv, &tdo, &tq16, &tk16, &tdq, q, k, o, o_lo, dout, v, lse, mask->row_cnt, mask->row_idx, mask->col_cnt,
-            mask->col_idx, w.dvec, w.do16, w.v16, w.q16, w.k16, dq, dk, dv, f32 ? 1 : 0, (int)s.BH, s.N, s.Tm, s.Tn, scale,
+  const int *rc = mask->row_cnt, *ri = mask->row_idx, *cc = mask->col_cnt, *ci = mask->col_idx;
+  if (s.tiled) {
+    SPA2_CUDA_TRY(launch_tile_lists(mask->row_cnt, mask->row_idx, mask->col_cnt, mask->col_idx, (int)s.BH, s.Tm, s.Tn,
+                                    s.TMt, s.TNt, s.bq, s.bkv, w.tiles.csr_cnt, w.tiles.csr_idx, w.tiles.csc_cnt,
+                                    w.tiles.csc_idx, w.status, st));
+    rc = w.tiles.csr_cnt;
+    ri = w.tiles.csr_idx;
+    cc = w.tiles.csc_cnt;
+    ci = w.tiles.csc_idx;
+  }
+  BwdArgs a{&tq, &tk, &tv, &tdo, &tq16, &tk16, &tdq, q, k, o, o_lo, dout, v, lse, rc, ri, cc, ci, w.dvec, w.do16,
+            w.v16, w.q16, w.k16, dq, dk, dv, f32 ? 1 : 0, (int)s.BH, s.N, s.TMt, s.TNt, scale,
             scale * 1.4426950408889634f, w.status, g_wait_limit_ns};
   SPA2_CUDA_TRY(launch_bwd(a, d, st));
   return SPA2_OK;

@@ -165,8 +165,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
       for (int t = 0; t < n; ++t) {
         const int s = t & 1;
         if (t >= 2 && !wait_bar(&sm.qd_empty[s], ((t >> 1) - 1) & 1, wc)) break;
-        const int i = q_list[t];
-        if (i < 0 || i >= Tm) {
+        const int i = q_list[t] & TILE_ID_MASK;
+        if (i >= Tm) {
           report(status, SPA2_ERR_DEVICE_BOUNDS);
           sm.abort_flag = 1;
           break;
@@ -267,7 +267,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
     // lse / D of the next tile's row, loaded a tile ahead
     float lse_n = INFINITY, d_n = 0.f;
     if (n > 0) {
-      const long long row = (long long)q_list[0] * 128 + r;
+      const long long row = (long long)(q_list[0] & TILE_ID_MASK) * 128 + r;
       if (row < N) {
         lse_n = lse[(long long)bh * N + row];
         d_n = dvec[(long long)bh * N + row];
@@ -277,7 +277,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
       const int s = t & 1;
       const float nlse2 = -lse_n * LOG2E, Dr = d_n;
       if (t + 1 < n) {
-        const long long row = (long long)q_list[t + 1] * 128 + r;
+        const long long row = (long long)(q_list[t + 1] & TILE_ID_MASK) * 128 + r;
         lse_n = row < N ? lse[(long long)bh * N + row] : INFINITY;
         d_n = row < N ? dvec[(long long)bh * N + row] : 0.f;
       }
@@ -292,6 +292,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
         break;
       }
       const uint64_t nlse2x2 = f2_pack(nlse2, nlse2), d2 = f2_pack(Dr, Dr);
+      // this row's half excluded (a 64-row query block that does not keep kv tile j)
+      const bool excl = tile_excluded(q_list[t], r >> 6);
 #pragma unroll
       for (int sub = 0; sub < 2; ++sub) {
         const int c0 = h * 32 + sub * 16;  // first kv column of this 16-column slice
@@ -311,6 +313,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
             if (c0 + 2 * e >= kv_valid) p0 = 0.f;
             if (c0 + 2 * e + 1 >= kv_valid) p1 = 0.f;
           }
+          if (excl) p0 = p1 = 0.f;
           pk[e] = pack_f16(p0, p1);
           const uint64_t ds2 = f2_mul(f2_pack(p0, p1),
                                       f2_sub(f2_pack(__uint_as_float(pa[2 * e]), __uint_as_float(pa[2 * e + 1])), d2));
@@ -487,8 +490,8 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_cons
       for (int t = 0; t < n; ++t) {
         const int slot = t % DQ_KS;
         if (t >= DQ_KS && !wait_bar(&sm.kv_empty[slot], ((t / DQ_KS) - 1) & 1, wc)) break;
-        const int j = kv_list[t];
-        if (j < 0 || j >= Tn) {
+        const int j = kv_list[t] & TILE_ID_MASK;
+        if (j >= Tn) {
           report(status, SPA2_ERR_DEVICE_BOUNDS);
           sm.abort_flag = 1;
           break;
@@ -580,7 +583,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_cons
     const uint64_t scale2 = f2_pack(scale_log2, scale_log2), nlse2x2 = f2_pack(nlse2, nlse2),
                    d2 = f2_pack(Dr, Dr);
     // only kv-block Tn-1 (last in the ascending list) is ragged
-    const int last_valid = (n > 0 && kv_list[n - 1] == Tn - 1) ? N - (Tn - 1) * 64 : 64;
+    const int last_valid = (n > 0 && (kv_list[n - 1] & TILE_ID_MASK) == Tn - 1) ? N - (Tn - 1) * 64 : 64;
     bool ok = n > 0;
     for (int t = 0; t < n && ok; ++t) {
       const int b = t & 1;
@@ -589,7 +592,8 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_cons
         break;
       }
       tc_fence_after();
-      const int kv_valid = t == n - 1 ? last_valid : 64;
+      // a tile excluded for this row's half contributes nothing (P = 0, dS = 0)
+      const int kv_valid = tile_excluded(kv_list[t], r >> 6) ? 0 : t == n - 1 ? last_valid : 64;
       const int c0 = h * 32;
       uint32_t sa[32], pa[32];
       tmem_ld32(tl + T_S + b * 64 + c0, sa);

@@ -123,8 +123,8 @@ __global__ void __launch_bounds__(192, 2) fwd_kernel(const __grid_constant__ CUt
       for (int t = 0; t < n; ++t) {
         const int s = t & 1;
         if (t >= 2 && !wait_bar(&sm.kv_empty[s], ((t >> 1) - 1) & 1, wc)) break;
-        const int j = kv_list[t];
-        if (j < 0 || j >= Tn) {
+        const int j = kv_list[t] & TILE_ID_MASK;
+        if (j >= Tn) {
           report(status, SPA2_ERR_DEVICE_BOUNDS);
           sm.abort_flag = 1;
           break;
@@ -187,8 +187,9 @@ __global__ void __launch_bounds__(192, 2) fwd_kernel(const __grid_constant__ CUt
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
     float m_use = -INFINITY, l = 0.f;
     bool ok = n > 0;
-    // only the kv-block Tn-1 is ragged, and the ascending list holds it last
-    const int last_valid = (n > 0 && kv_list[n - 1] == Tn - 1) ? (N - (Tn - 1) * 64) : 64;
+    // only the kv tile Tn-1 is ragged, and the ascending list holds it last
+    const int last_valid = (n > 0 && (kv_list[n - 1] & TILE_ID_MASK) == Tn - 1) ? (N - (Tn - 1) * 64) : 64;
+    const int half = warp >> 1;  // rows 64*half .. 64*half+63 of the tile
     for (int t = 0; t < n && ok; ++t) {
       const int s = t & 1;
       if (!wait_warp(&sm.s_full[s], (t >> 1) & 1, wc)) {
@@ -196,7 +197,10 @@ __global__ void __launch_bounds__(192, 2) fwd_kernel(const __grid_constant__ CUt
         break;
       }
       tc_fence_after();
-      const int valid = (t == n - 1) ? last_valid : 64;
+      // a tile excluded for this row's half (a 64-row query block that does not
+      // keep it) contributes nothing: every logit masked
+      const bool excl = tile_excluded(kv_list[t], half);
+      const int valid = excl ? 0 : (t == n - 1) ? last_valid : 64;
       uint32_t sv[64];
       tmem_ld64(tl + s * 64, sv);
       tmem_wait_ld();
@@ -224,7 +228,7 @@ __global__ void __launch_bounds__(192, 2) fwd_kernel(const __grid_constant__ CUt
         l *= alpha;
         rescale = true;
       }
-      const float neg_m = -m_use;
+      const float neg_m = m_use == -INFINITY ? 0.f : -m_use;  // nothing seen yet: every P is 0
       uint32_t pk[32];
       float rsum[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll

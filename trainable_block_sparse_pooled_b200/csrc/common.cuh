@@ -450,6 +450,18 @@ SPA2_DEV uint64_t f2_mul(uint64_t a, uint64_t b) {
   return r;
 }
 
+// ---------------------------------------------------------------------------
+// Tile lists. The attention kernels work on tiles of 128 query rows x 64 key
+// rows and read, per query tile (forward, dQ) or key tile (dK/dV), a list of
+// the tiles it meets. An entry is a tile id in bits 0-29; bit 30 (31) set
+// means rows 0-63 (64-127) of the 128-row query tile are excluded from it,
+// which happens when 64-row query blocks share a tile but keep different
+// key blocks. With 128-row query blocks and 64-row key blocks the block CSR /
+// CSC are the tile lists as they are (no bit set).
+// ---------------------------------------------------------------------------
+constexpr int TILE_ID_MASK = 0x3FFFFFFF;
+SPA2_DEV bool tile_excluded(int entry, int half) { return ((unsigned)entry >> (30 + half)) & 1u; }
+
 SPA2_DEV float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -20,6 +20,7 @@ enum KernelId : int {
   KID_BWD_DKDV,
   KID_BWD_DQ,
   KID_PROBE,
+  KID_TILES,
   KID_COUNT
 };
 
@@ -115,5 +116,11 @@ cudaError_t launch_bwd(const BwdArgs& a, int d, cudaStream_t s);
 
 // api.cu
 cudaError_t launch_timeout_probe(int* status, unsigned long long limit_ns, cudaStream_t s);
+
+// tiles.cu: block CSR (and CSC when csc_cnt is not NULL) -> tile lists of 128-row query tiles x 64-row key
+// tiles (TMt = ceil(N / 128), TNt = ceil(N / 64)); see the tile-list notes in common.cuh
+cudaError_t launch_tile_lists(const int* row_cnt, const int* row_idx, const int* col_cnt, const int* col_idx, int BH,
+                              int Tm, int Tn, int TMt, int TNt, int bq, int bkv, int* csr_cnt, int* csr_idx,
+                              int* csc_cnt, int* csc_idx, int* status, cudaStream_t s);
 
 }  // namespace spa2

@@ -25,6 +25,7 @@ const char* const kNames[KID_COUNT] = {
     "bwd_dkdv_kernel",    // KID_BWD_DKDV
     "bwd_dq_kernel",      // KID_BWD_DQ
     "timeout_probe_kernel",  // KID_PROBE
+    "tile_list_kernel",   // KID_TILES
 };
 
 struct Record {
