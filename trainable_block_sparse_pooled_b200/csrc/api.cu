@@ -106,7 +106,7 @@ static size_t tile_ws(char* base, size_t off, const Shape& s, bool csc, TileWs* 
 
 struct FwdWs {
   int* status;
-  void* v16;
+  void* v16;  // fp16 copy of V [BH, N, d]
   TileWs tiles;
   size_t bytes;
 };
@@ -368,9 +368,8 @@ spa2_status spa2_sparse_attn_fwd(const void* q, const void* k, const void* v, in
   if (ws_bytes < w.bytes) return SPA2_ERR_WORKSPACE;
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)d);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  void* v16 = w.v16;
   CUtensorMap tq, tk, tv, to, tolo;
-  if (!make_map(&tq, q, s, 128) || !make_map(&tk, k, s, 64) || !make_map(&tv, v16, s, 64, true) ||
+  if (!make_map(&tq, q, s, 128) || !make_map(&tk, k, s, 64) || !make_map(&tv, w.v16, s, 64, true) ||
       !make_map(&to, o, s, 128) || !make_map(&tolo, o_lo ? o_lo : o, s, 128))
     return SPA2_ERR_CUDA;
   int* status = w.status;
@@ -384,9 +383,9 @@ spa2_status spa2_sparse_attn_fwd(const void* q, const void* k, const void* v, in
     rc = w.tiles.csr_cnt;
     ri = w.tiles.csr_idx;
   }
-  SPA2_CUDA_TRY(launch_v_to_f16(v, v16, s.BH * s.N * s.d, status, st));
+  SPA2_CUDA_TRY(launch_v_to_f16(v, w.v16, s.BH * s.N * s.d, status, st));
   FwdArgs a{&tq, &tk, &tv, &to, &tolo, o_lo != nullptr, rc, ri, lse, (int)s.BH, s.N, s.TMt, s.TNt,
-            scale * 1.4426950408889634f, status, g_wait_limit_ns};
+            scale * 1.4426950408889634f, status, g_wait_limit_ns, s.tiled ? 1 : 0};
   SPA2_CUDA_TRY(launch_fwd(a, d, st));
   return SPA2_OK;
 }
@@ -430,7 +429,7 @@ spa2_status spa2_sparse_attn_bwd(const void* q, const void* k, const void* v, co
   }
   BwdArgs a{&tq, &tk, &tv, &tdo, &tq16, &tk16, &tdq, q, k, o, o_lo, dout, v, lse, rc, ri, cc, ci, w.dvec, w.do16,
             w.v16, w.q16, w.k16, dq, dk, dv, f32 ? 1 : 0, (int)s.BH, s.N, s.TMt, s.TNt, scale,
-            scale * 1.4426950408889634f, w.status, g_wait_limit_ns};
+            scale * 1.4426950408889634f, w.status, g_wait_limit_ns, s.tiled ? 1 : 0};
   SPA2_CUDA_TRY(launch_bwd(a, d, st));
   return SPA2_OK;
 }

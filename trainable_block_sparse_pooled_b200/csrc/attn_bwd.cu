@@ -82,7 +82,8 @@ SPA2_DEV void split_bf16(float a, float b, uint32_t& hi, uint32_t& lo) {
 
 }  // namespace
 
-template <int D>
+// TILED: list entries may carry exclusion bits (block sizes other than (128, 64))
+template <int D, bool TILED>
 __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q16,
                                                                   const __grid_constant__ CUtensorMap tm_k16,
                                                                   const __grid_constant__ CUtensorMap tm_v16,
@@ -293,7 +294,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
       }
       const uint64_t nlse2x2 = f2_pack(nlse2, nlse2), d2 = f2_pack(Dr, Dr);
       // this row's half excluded (a 64-row query block that does not keep kv tile j)
-      const bool excl = tile_excluded(q_list[t], r >> 6);
+      const bool excl = TILED && tile_excluded(q_list[t], r >> 6);
 #pragma unroll
       for (int sub = 0; sub < 2; ++sub) {
         const int c0 = h * 32 + sub * 16;  // first kv column of this 16-column slice
@@ -416,7 +417,7 @@ struct DqSmem {
 // 128 bytes per cycle the tensor core can read from shared memory).
 // TMEM columns: S[b] 64b .. 64b+63 (dS hi/lo of kv columns 32h .. 32h+31 go to
 // 64b+32h .. +15 / +16 .. +31), dP[b] 128+64b, dQ 256 .. 256+d, Q 384, dO 448.
-template <int D>
+template <int D, bool TILED>
 __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k,
                                                                const __grid_constant__ CUtensorMap tm_v16,
                                                                const __grid_constant__ CUtensorMap tm_dq,
@@ -593,7 +594,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_cons
       }
       tc_fence_after();
       // a tile excluded for this row's half contributes nothing (P = 0, dS = 0)
-      const int kv_valid = tile_excluded(kv_list[t], r >> 6) ? 0 : t == n - 1 ? last_valid : 64;
+      const int kv_valid = (TILED && tile_excluded(kv_list[t], r >> 6)) ? 0 : t == n - 1 ? last_valid : 64;
       const int c0 = h * 32;
       uint32_t sa[32], pa[32];
       tmem_ld32(tl + T_S + b * 64 + c0, sa);
@@ -749,7 +750,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __res
   if (bad) report(status, SPA2_ERR_RANGE);
 }
 
-template <int D>
+template <int D, bool TILED>
 static cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
   const long long rows = (long long)a.BH * a.N;
   // 1. D and the fp16 copies of dO and V
@@ -766,10 +767,10 @@ static cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
   // 2. dK, dV (kv-major)
   {
     const size_t smem = sizeof(BwdSmem<D>) + 1024;
-    e = cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(bwd_dkdv_kernel<D, TILED>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     KernelTimer kt(KID_BWD_DKDV, s);
-    bwd_dkdv_kernel<D><<<dim3(a.Tn, a.BH), BWD_THREADS, smem, s>>>(
+    bwd_dkdv_kernel<D, TILED><<<dim3(a.Tn, a.BH), BWD_THREADS, smem, s>>>(
         *a.tm_q16, *a.tm_k16, *a.tm_v, *a.tm_do, a.lse, a.dvec, a.col_cnt, a.col_idx, a.dk, a.dv, a.grad_f32, a.N, a.Tm,
         a.Tn, a.scale, a.scale_log2, a.status, a.wait_limit_ns);
     e = cudaGetLastError();
@@ -778,10 +779,10 @@ static cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
   // 3. dQ (q-major)
   {
     const size_t smem = sizeof(DqSmem<D>) + 1024;
-    e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(bwd_dq_kernel<D, TILED>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     KernelTimer kt(KID_BWD_DQ, s);
-    bwd_dq_kernel<D><<<dim3(a.Tm, a.BH), DQ_THREADS, smem, s>>>(
+    bwd_dq_kernel<D, TILED><<<dim3(a.Tm, a.BH), DQ_THREADS, smem, s>>>(
         *a.tm_k, *a.tm_v, *a.tm_dq, static_cast<const __nv_bfloat16*>(a.q), static_cast<const __half*>(a.do16),
         a.lse, a.dvec, a.row_cnt, a.row_idx, a.grad_f32, a.N, a.Tm, a.Tn, a.scale, a.scale_log2, a.status,
         a.wait_limit_ns);
@@ -791,7 +792,8 @@ static cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_bwd(const BwdArgs& a, int d, cudaStream_t s) {
-  return d == 128 ? launch_bwd_d<128>(a, s) : launch_bwd_d<64>(a, s);
+  if (d == 128) return a.tiled ? launch_bwd_d<128, true>(a, s) : launch_bwd_d<128, false>(a, s);
+  return a.tiled ? launch_bwd_d<64, true>(a, s) : launch_bwd_d<64, false>(a, s);
 }
 
 }  // namespace spa2

@@ -5,7 +5,9 @@
 // One CTA per (q-block i, head): 128 query rows (b_q = 128) against the kept
 // kv-blocks j (b_kv = 64 rows each) listed in the CSR row of i.
 //
-//   warp 4      TMA producer: Q_i once, then K_j / V_j through a 2-slot ring.
+//   warp 4      TMA producer: Q_i once, then K_j and V_j through 2-slot rings;
+//               a K slot is refilled as soon as its S product is done, a V slot
+//               once its P V product is done (whichever is free first).
 //   warp 5      MMA issuer (all 32 lanes run the loop, elect.sync picks the lane
 //               that issues each tcgen05 op): S = Q K_j^T (SS, bf16, M=128 N=64 K=d)
 //               into one of two TMEM S buffers; O += P V_j (TS: P from TMEM,
@@ -39,7 +41,7 @@ struct FwdSmem {
   alignas(1024) uint8_t k[2][CH][64 * 128];
   alignas(1024) uint8_t v[2][CH][64 * 128];
   uint64_t q_full;
-  uint64_t k_full[2], v_full[2], kv_empty[2];
+  uint64_t k_full[2], v_full[2], k_empty[2], v_empty[2];
   uint64_t s_full[2], p_full[2], o_done, drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -54,7 +56,9 @@ SPA2_DEV bool wait_warp(uint64_t* bar, uint32_t parity, const WaitCtx& w) {
 
 }  // namespace
 
-template <int D>
+// TILED: the list entries may carry exclusion bits (block sizes other than
+// (128, 64)); without it they are plain ids and no check is compiled in
+template <int D, bool TILED>
 __global__ void __launch_bounds__(192, 2) fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                      const __grid_constant__ CUtensorMap tm_k,
                                                      const __grid_constant__ CUtensorMap tm_v,
@@ -87,7 +91,8 @@ __global__ void __launch_bounds__(192, 2) fwd_kernel(const __grid_constant__ CUt
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.k_full[s], 1);
       mbar_init(&sm.v_full[s], 1);
-      mbar_init(&sm.kv_empty[s], 1);
+      mbar_init(&sm.k_empty[s], 1);
+      mbar_init(&sm.v_empty[s], 1);
       mbar_init(&sm.s_full[s], 1);
       mbar_init(&sm.p_full[s], 128);
     }
@@ -119,28 +124,55 @@ __global__ void __launch_bounds__(192, 2) fwd_kernel(const __grid_constant__ CUt
       tma_prefetch_desc(&tm_v);
       mbar_expect_tx(&sm.q_full, Q_BYTES);
       for (int c = 0; c < CH; ++c) tma_load_3d(sm.q[c], &tm_q, &sm.q_full, c * 64, i * 128, bh);
-      int issued = 0;
-      for (int t = 0; t < n; ++t) {
-        const int s = t & 1;
-        if (t >= 2 && !wait_bar(&sm.kv_empty[s], ((t >> 1) - 1) & 1, wc)) break;
-        const int j = kv_list[t] & TILE_ID_MASK;
-        if (j >= Tn) {
-          report(status, SPA2_ERR_DEVICE_BOUNDS);
-          sm.abort_flag = 1;
-          break;
+      // the fp16 copy of V comes from the kernel launched just before this one
+      pdl_wait();
+      // K(kt) needs S(kt - 2) done, V(vt) needs P V(vt - 2) done; take whichever
+      // is free, K first (its product comes first)
+      int kt = 0, vt = 0;
+      uint64_t t0 = 0;
+      uint32_t idle = 0;
+      while (vt < n) {
+        if (kt < n && (kt < 2 || mbar_test_wait(&sm.k_empty[kt & 1], ((kt >> 1) - 1) & 1))) {
+          const int j = kv_list[kt] & TILE_ID_MASK;
+          if (j >= Tn) {
+            report(status, SPA2_ERR_DEVICE_BOUNDS);
+            sm.abort_flag = 1;
+            break;
+          }
+          mbar_expect_tx(&sm.k_full[kt & 1], KV_BYTES);
+          for (int c = 0; c < CH; ++c) tma_load_3d(sm.k[kt & 1][c], &tm_k, &sm.k_full[kt & 1], c * 64, j * 64, bh);
+          ++kt;
+          idle = 0;
+          t0 = 0;
+        } else if (vt < kt && (vt < 2 || mbar_test_wait(&sm.v_empty[vt & 1], ((vt >> 1) - 1) & 1))) {
+          const int j = kv_list[vt] & TILE_ID_MASK;
+          mbar_expect_tx(&sm.v_full[vt & 1], KV_BYTES);
+          for (int c = 0; c < CH; ++c) tma_load_3d(sm.v[vt & 1][c], &tm_v, &sm.v_full[vt & 1], c * 64, j * 64, bh);
+          ++vt;
+          idle = 0;
+          t0 = 0;
+        } else {
+          // nothing free: sleep in try_wait on the slot that frees next, not a hot spin
+          if (kt < n && kt >= 2)
+            mbar_try_wait(&sm.k_empty[kt & 1], ((kt >> 1) - 1) & 1);
+          else if (vt < kt && vt >= 2)
+            mbar_try_wait(&sm.v_empty[vt & 1], ((vt >> 1) - 1) & 1);
+          if ((++idle & 63u) != 0u) continue;
+          if (sm.abort_flag) break;
+          const uint64_t now = globaltimer_ns();
+          if (t0 == 0) {
+            t0 = now;
+          } else if (now - t0 > wait_limit_ns) {
+            report(status, SPA2_ERR_DEVICE_TIMEOUT);
+            sm.abort_flag = 1;
+            break;
+          }
         }
-        mbar_expect_tx(&sm.k_full[s], KV_BYTES);
-        for (int c = 0; c < CH; ++c) tma_load_3d(sm.k[s][c], &tm_k, &sm.k_full[s], c * 64, j * 64, bh);
-        mbar_expect_tx(&sm.v_full[s], KV_BYTES);
-        for (int c = 0; c < CH; ++c) tma_load_3d(sm.v[s][c], &tm_v, &sm.v_full[s], c * 64, j * 64, bh);
-        issued = t + 1;
       }
       // never leave with copies in flight: wait (bounded) for the last loads
       const WaitCtx drain_wc{&sm.never, nullptr, wait_limit_ns};
-      for (int t = max(0, issued - 2); t < issued; ++t) {
-        wait_bar(&sm.k_full[t & 1], (t >> 1) & 1, drain_wc);
-        wait_bar(&sm.v_full[t & 1], (t >> 1) & 1, drain_wc);
-      }
+      for (int t = max(0, kt - 2); t < kt; ++t) wait_bar(&sm.k_full[t & 1], (t >> 1) & 1, drain_wc);
+      for (int t = max(0, vt - 2); t < vt; ++t) wait_bar(&sm.v_full[t & 1], (t >> 1) & 1, drain_wc);
       wait_bar(&sm.q_full, 0, drain_wc);
     }
   } else if (warp == 5) {
@@ -160,6 +192,7 @@ __global__ void __launch_bounds__(192, 2) fwd_kernel(const __grid_constant__ CUt
               mma_ss_el(tmem + s * 64, a, b, IDESC_S, kk > 0 ? 1u : 0u);
             }
             mma_commit_el(&sm.s_full[s]);
+            mma_commit_el(&sm.k_empty[s]);
           }
           if (t >= 1) {
             const int u = t - 1, su = u & 1;
@@ -171,7 +204,7 @@ __global__ void __launch_bounds__(192, 2) fwd_kernel(const __grid_constant__ CUt
               const uint64_t b = sdesc_sw128(smem_u32(sm.v[su][0]) + kk * 2048, 64 * 128, 1024);
               mma_ts_el(tmem_o, tmem + su * 64 + kk * 8, b, IDESC_O, (u > 0 || kk > 0) ? 1u : 0u);
             }
-            mma_commit_el(&sm.kv_empty[su]);
+            mma_commit_el(&sm.v_empty[su]);
             mma_commit_el(&sm.o_done);
           }
         }
@@ -199,7 +232,7 @@ __global__ void __launch_bounds__(192, 2) fwd_kernel(const __grid_constant__ CUt
       tc_fence_after();
       // a tile excluded for this row's half (a 64-row query block that does not
       // keep it) contributes nothing: every logit masked
-      const bool excl = tile_excluded(kv_list[t], half);
+      const bool excl = TILED && tile_excluded(kv_list[t], half);
       const int valid = excl ? 0 : (t == n - 1) ? last_valid : 64;
       uint32_t sv[64];
       tmem_ld64(tl + s * 64, sv);
@@ -323,6 +356,7 @@ __global__ void __launch_bounds__(192, 2) fwd_kernel(const __grid_constant__ CUt
 // to the largest finite fp16 and reported as SPA2_ERR_RANGE.
 __global__ void __launch_bounds__(256) v_to_f16_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
                                                        long long n8, int* status) {
+  pdl_trigger();  // the forward kernel may start its prologue (Q load, TMEM, barriers)
   bool bad = false;
   for (long long e = (long long)blockIdx.x * 256 + threadIdx.x; e < n8; e += (long long)gridDim.x * 256) {
     const uint4 v = src[e];
@@ -347,27 +381,24 @@ cudaError_t launch_v_to_f16(const void* v, void* v16, long long elems, int* stat
   const long long n8 = elems / 8;
   const unsigned blocks = (unsigned)((n8 + 255) / 256 < 148LL * 32 ? (n8 + 255) / 256 : 148LL * 32);
   KernelTimer kt(KID_V16, s);
-  v_to_f16_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4*>(v), static_cast<uint4*>(v16), n8, status);
-  return cudaGetLastError();
+  return launch_k(v_to_f16_kernel, dim3(blocks), dim3(256), 0, s, false, static_cast<const uint4*>(v),
+                  static_cast<uint4*>(v16), n8, status);
+}
+
+template <int D, bool TILED>
+static cudaError_t launch_fwd_t(const FwdArgs& a, cudaStream_t s) {
+  const size_t smem = sizeof(FwdSmem<D>) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(fwd_kernel<D, TILED>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  return launch_k(fwd_kernel<D, TILED>, dim3(a.Tm, a.BH), dim3(192), smem, s, true, *a.tm_q, *a.tm_k, *a.tm_v,
+                  *a.tm_o, *a.tm_olo, a.has_olo, a.row_cnt, a.row_idx, a.lse, a.N, a.Tm, a.Tn, a.scale_log2, a.status,
+                  a.wait_limit_ns);
 }
 
 cudaError_t launch_fwd(const FwdArgs& a, int d, cudaStream_t s) {
-  dim3 grid(a.Tm, a.BH);
   KernelTimer kt(KID_FWD, s);
-  if (d == 128) {
-    const size_t smem = sizeof(FwdSmem<128>) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    fwd_kernel<128><<<grid, 192, smem, s>>>(*a.tm_q, *a.tm_k, *a.tm_v, *a.tm_o, *a.tm_olo, a.has_olo, a.row_cnt, a.row_idx, a.lse, a.N,
-                                            a.Tm, a.Tn, a.scale_log2, a.status, a.wait_limit_ns);
-  } else {
-    const size_t smem = sizeof(FwdSmem<64>) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    fwd_kernel<64><<<grid, 192, smem, s>>>(*a.tm_q, *a.tm_k, *a.tm_v, *a.tm_o, *a.tm_olo, a.has_olo, a.row_cnt, a.row_idx, a.lse, a.N,
-                                           a.Tm, a.Tn, a.scale_log2, a.status, a.wait_limit_ns);
-  }
-  return cudaGetLastError();
+  if (d == 128) return a.tiled ? launch_fwd_t<128, true>(a, s) : launch_fwd_t<128, false>(a, s);
+  return a.tiled ? launch_fwd_t<64, true>(a, s) : launch_fwd_t<64, false>(a, s);
 }
 
 }  // namespace spa2

@@ -73,6 +73,7 @@ struct FwdArgs {
   float scale_log2;   // softmax_scale * log2(e)
   int* status;
   unsigned long long wait_limit_ns;
+  int tiled;          // list entries may carry tile exclusion bits
 };
 cudaError_t launch_fwd(const FwdArgs& a, int d, cudaStream_t s);
 cudaError_t launch_v_to_f16(const void* v, void* v16, long long elems, int* status, cudaStream_t s);
@@ -111,6 +112,7 @@ struct BwdArgs {
   float scale_log2;   // softmax_scale * log2(e)
   int* status;
   unsigned long long wait_limit_ns;
+  int tiled;          // list entries may carry tile exclusion bits
 };
 cudaError_t launch_bwd(const BwdArgs& a, int d, cudaStream_t s);
 
