@@ -58,8 +58,8 @@ static bool frac_ok(float x) { return x >= 0.f && x <= 1.f; }  // false for NaN
 // workspace layout -----------------------------------------------------------
 struct MaskWs {
   int* status;
-  float* qbar;  // Qbar [BH, Tm, d]
-  float* kbT;   // Kbar^T [BH, d, kbar_cols(Tn)]
+  float* qbar;  // Qbar in 64-row chunks [BH, kbar_chunks(Tm), d, 64]
+  float* kbc;   // Kbar in 64-key chunks [BH, kbar_chunks(Tn), d, 64]
   float* lg;    // pooled logits [BH, Tm, Tn]
   uint32_t* bits;
   size_t bytes;
@@ -70,9 +70,9 @@ static MaskWs mask_ws(void* ws, const Shape& s) {
   char* base = static_cast<char*>(ws);
   w.status = reinterpret_cast<int*>(base);
   w.qbar = reinterpret_cast<float*>(base + off);
-  off += al256((size_t)s.BH * s.Tm * s.d * 4);
-  w.kbT = reinterpret_cast<float*>(base + off);
-  off += al256((size_t)s.BH * s.d * kbar_cols(s.Tn) * 4);
+  off += al256((size_t)s.BH * kbar_chunks(s.Tm) * s.d * 64 * 4);
+  w.kbc = reinterpret_cast<float*>(base + off);
+  off += al256((size_t)s.BH * kbar_chunks(s.Tn) * s.d * 64 * 4);
   w.lg = reinterpret_cast<float*>(base + off);
   off += al256((size_t)s.BH * s.Tm * s.Tn * 4);
   w.bits = reinterpret_cast<uint32_t*>(base + off);
@@ -324,7 +324,7 @@ spa2_status spa2_block_mask(const void* q, const void* k, int B, int H, int N, i
 
   SPA2_CUDA_TRY(cudaMemsetAsync(w.status, 0, 4, st));
   MaskOut mo{out->row_cnt, out->row_idx, out->pbar, out->bitmap};
-  SPA2_CUDA_TRY(launch_mask(q, k, w.qbar, w.kbT, w.lg, (int)s.BH, s.N, s.d, s.Tm, s.Tn, bq, bkv, topk_count(k_frac, s.Tn),
+  SPA2_CUDA_TRY(launch_mask(q, k, w.qbar, w.kbc, w.lg, (int)s.BH, s.N, s.d, s.Tm, s.Tn, bq, bkv, topk_count(k_frac, s.Tn),
                             topp_threshold(p_frac), mo, out->col_cnt, out->col_idx, w.bits, s.W, w.status,
                             g_wait_limit_ns, st));
   return SPA2_OK;

@@ -46,10 +46,11 @@ struct MaskOut {
 };
 
 // mask.cu
-// qbar: Qbar workspace [BH, Tm, d] fp32; kbT: Kbar^T workspace [BH, d, kbar_cols(Tn)] fp32;
+// qbar, kbc: Qbar and Kbar workspaces in chunks of 64 blocks,
+// [BH, kbar_chunks(Tm), d, 64] and [BH, kbar_chunks(Tn), d, 64] fp32;
 // lg: logit workspace [BH, Tm, Tn] fp32
-int kbar_cols(int Tn);
-cudaError_t launch_mask(const void* q, const void* k, float* qbar, float* kbT, float* lg, int BH, int N, int d,
+int kbar_chunks(int Tn);
+cudaError_t launch_mask(const void* q, const void* k, float* qbar, float* kbc, float* lg, int BH, int N, int d,
                         int Tm, int Tn, int bq, int bkv, int K, unsigned long long thr, const MaskOut& out,
                         int* col_cnt, int* col_idx, uint32_t* bits, int W, int* status,
                         unsigned long long wait_limit_ns, cudaStream_t s);

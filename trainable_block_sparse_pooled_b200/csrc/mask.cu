@@ -2,14 +2,14 @@
 // 方法步骤详情 steps 1-3; 技术新颖性 union formula; gist.science 2A).
 //
 //   pool_kernel    one CTA per block, every streaming load of a thread in flight
-//                  before it sums: means of the q-blocks -> Qbar
-//                  [B*H, T_m, d] and of the kv-blocks -> Kbar^T [B*H, d, T_n']
-//                  fp32 (transposed, T_n' = T_n rounded up to a multiple of 4,
-//                  so the logit loop reads the keys of one feature with
-//                  coalesced 8-byte loads).
-//   logits_kernel  S-bar = Qbar Kbar^T / sqrt(d), fp32, by CTAs of 16 rows x 128
-//                  keys of one head (thread = pair of keys against 4 rows) ->
-//                  logit scratch [B*H, T_m, T_n].
+//                  before it sums: means of the q-blocks and kv-blocks -> Qbar
+//                  and Kbar in chunks of 64 blocks, each chunk d x 64
+//                  ([B*H, ceil(T_m / 64), d, 64], [B*H, ceil(T_n / 64), d, 64],
+//                  fp32).
+//   logits_kernel  S-bar = Qbar Kbar^T / sqrt(d), fp32: one CTA per 64 x 64 tile
+//                  of one head, both chunks by bulk copy into shared memory,
+//                  thread = 4 rows x 4 keys with paired fp32 FMAs -> logit
+//                  scratch [B*H, T_m, T_n].
 //   select_kernel  one warp per row, the row in registers: softmax -> P-bar,
 //                  hybrid selection -> CSR, kept-bit words, optional P-bar /
 //                  uint8 bitmap.
@@ -431,15 +431,17 @@ SPA2_DEV void csc_word_cta(const uint32_t* __restrict__ head_bits, int Tm, int T
 
 }  // namespace
 
+constexpr int LG_C = 64;  // rows (keys) per Qbar (Kbar) chunk: one logits tile is 64 x 64
+
 // Pooling: one CTA of 256 threads per block (blockIdx.x < T_m: q-block ->
-// Qbar row-major; otherwise kv-block -> Kbar^T column). Each thread owns a
+// Qbar; otherwise kv-block -> Kbar chunk column). Each thread owns a
 // 16-byte column chunk of every 16th (d = 128) or 32nd (d = 64) row and issues
 // all of its streaming loads of a 128-row span before summing; partial sums
 // meet in shared memory.
 template <int D>
 __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ q,
                                                    const __nv_bfloat16* __restrict__ k, float* __restrict__ qbar,
-                                                   float* __restrict__ kbT, int N, int Tm, int Tn, int TnP, int bq,
+                                                   float* __restrict__ kbc, int N, int Tm, int Tn, int bq,
                                                    int bkv) {
   constexpr int TPR = D / 8;        // threads per row (8 bf16 each)
   constexpr int RP = 256 / TPR;     // rows per pass
@@ -485,62 +487,98 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
     for (int i = 0; i < RP; ++i) sum += red[i * (D + 1) + threadIdx.x];
     const float mean = sum / static_cast<float>(rows);
     if (is_q)
-      qbar[(h * Tm + idx) * D + threadIdx.x] = mean;
+      qbar[((h * ((Tm + LG_C - 1) / LG_C) + (idx >> 6)) * D + threadIdx.x) * LG_C + (idx & 63)] = mean;
     else
-      kbT[(h * D + threadIdx.x) * TnP + idx] = mean;
+      kbc[((h * ((Tn + LG_C - 1) / LG_C) + (idx >> 6)) * D + threadIdx.x) * LG_C + (idx & 63)] = mean;
   }
 }
 
 // Pooled logits: S-bar = Qbar Kbar^T / sqrt(d) -> lg [B*H, Tm, Tn] fp32. CTA
-// (key block of 128, row group of 16, head): the 16 pooled rows go to shared
-// memory transposed ([d][16]); thread (key pair kp, quarter hq) accumulates
-// keys 2kp, 2kp+1 against rows 4hq .. 4hq+3, the keys read from Kbar^T with
-// coalesced 8-byte loads (the four quarters of a CTA read the same keys, the
-// later ones from L1), 16 in flight.
-constexpr int LG_ROWS = 16, LG_KEYS = 128;
+// (key chunk, row chunk, head) of 128 threads computes one 64 x 64 tile: both
+// chunks (d x 64 each) arrive by bulk copy; thread (ty, tx) holds rows
+// 8ty..8ty+7 x keys 4tx..4tx+3 and adds, for d in order, two 16-byte loads of
+// its rows (four row pairs) and one of its keys: four key-pair registers and
+// sixteen paired fp32 FMAs (two products each) per column, the loads of four
+// columns issued ahead of their FMAs; then scales by 1/sqrt(d).
+template <int D>
+struct LogitSmem {
+  static constexpr int CHUNK_BYTES = D * LG_C * 4;
+  static constexpr int TOTAL = 2 * CHUNK_BYTES;  // Kbar chunk, then Qbar chunk
+};
 
 template <int D>
-__global__ void __launch_bounds__(256) logits_kernel(const float* __restrict__ qbar, const float* __restrict__ kbT,
-                                                     float* __restrict__ lg, int Tm, int Tn, int TnP,
-                                                     float inv_sqrt_d) {
-  __shared__ __align__(16) float qs[D * LG_ROWS];
-  pdl_wait();     // Qbar and Kbar^T are complete
-  pdl_trigger();  // the select kernel may be scheduled; it waits for this grid itself
+__global__ void __launch_bounds__(128, 3) logits_kernel(const float* __restrict__ qbar, const float* __restrict__ kbc,
+                                                     float* __restrict__ lg, int Tm, int Tn, float inv_sqrt_d,
+                                                     int* status, unsigned long long wait_limit_ns) {
+  using L = LogitSmem<D>;
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  const float* ks = reinterpret_cast<const float*>(smem);
+  const float* qs = reinterpret_cast<const float*>(smem + L::CHUNK_BYTES);
+  const int c = blockIdx.x, C = gridDim.x, rq = blockIdx.y, CQ = gridDim.y;
   const long long h = blockIdx.z;
-  const int i0 = blockIdx.y * LG_ROWS;
-  const int rc = min(LG_ROWS, Tm - i0);
-  for (int x = threadIdx.x; x < LG_ROWS * D; x += 256) {
-    const int r = x / D, dd = x % D;
-    qs[dd * LG_ROWS + r] = r < rc ? qbar[(h * Tm + i0 + r) * D + dd] : 0.f;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
   }
   __syncthreads();
-  const int kp = (int)threadIdx.x & 63, hq = (int)threadIdx.x >> 6;
-  const int key = blockIdx.x * LG_KEYS + 2 * kp;
-  if (key >= Tn || hq * 4 >= rc) return;
-  float a0[4], a1[4];
-#pragma unroll
-  for (int r = 0; r < 4; ++r) a0[r] = a1[r] = 0.f;
-  const float2* kcol = reinterpret_cast<const float2*>(kbT + h * D * TnP + key);
-#pragma unroll 16
-  for (int dd = 0; dd < D; ++dd) {
-    const float2 kv = __ldg(kcol + (long long)dd * (TnP / 2));
-    const float4 qq = *reinterpret_cast<const float4*>(qs + dd * LG_ROWS + hq * 4);
-    a0[0] = fmaf(kv.x, qq.x, a0[0]);
-    a1[0] = fmaf(kv.y, qq.x, a1[0]);
-    a0[1] = fmaf(kv.x, qq.y, a0[1]);
-    a1[1] = fmaf(kv.y, qq.y, a1[1]);
-    a0[2] = fmaf(kv.x, qq.z, a0[2]);
-    a1[2] = fmaf(kv.y, qq.z, a1[2]);
-    a0[3] = fmaf(kv.x, qq.w, a0[3]);
-    a1[3] = fmaf(kv.y, qq.w, a1[3]);
+  pdl_wait();     // Qbar and Kbar are complete
+  pdl_trigger();  // the select kernel may be scheduled; it waits for this grid itself
+  if (threadIdx.x == 0) {
+    mbar_expect_tx(&bar, 2u * L::CHUNK_BYTES);
+    bulk_load(smem, kbc + (h * C + c) * D * LG_C, L::CHUNK_BYTES, &bar);
+    bulk_load(smem + L::CHUNK_BYTES, qbar + (h * CQ + rq) * D * LG_C, L::CHUNK_BYTES, &bar);
   }
+  const WaitCtx wc{&abort_flag, status, wait_limit_ns};
+  wait_bar(&bar, 0, wc);
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+  uint64_t acc[4][4];  // [row pair][key]: {row 8ty + 2p, row 8ty + 2p + 1}
 #pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const int row = hq * 4 + r;
-    if (row < rc) {
-      float* dst = lg + (h * Tm + i0 + row) * Tn + key;
-      dst[0] = a0[r] * inv_sqrt_d;
-      if (key + 1 < Tn) dst[1] = a1[r] * inv_sqrt_d;
+  for (int p = 0; p < 4; ++p)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[p][j] = 0ull;
+  const ulonglong2* qrow = reinterpret_cast<const ulonglong2*>(qs) + 2 * ty;  // column dd at qrow[dd * 16], +1
+  const float4* kcol = reinterpret_cast<const float4*>(ks) + tx;              // column dd at kcol[dd * 16]
+#pragma unroll 1
+  for (int d0 = 0; d0 < D; d0 += 4) {
+    ulonglong2 qa[4], qb[4];
+    float4 kv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      qa[u] = qrow[(d0 + u) * (LG_C / 4)];
+      qb[u] = qrow[(d0 + u) * (LG_C / 4) + 1];
+      kv[u] = kcol[(d0 + u) * (LG_C / 4)];
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint64_t kk[4] = {f2_pack(kv[u].x, kv[u].x), f2_pack(kv[u].y, kv[u].y), f2_pack(kv[u].z, kv[u].z),
+                              f2_pack(kv[u].w, kv[u].w)};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        acc[0][j] = f2_fma(qa[u].x, kk[j], acc[0][j]);
+        acc[1][j] = f2_fma(qa[u].y, kk[j], acc[1][j]);
+        acc[2][j] = f2_fma(qb[u].x, kk[j], acc[2][j]);
+        acc[3][j] = f2_fma(qb[u].y, kk[j], acc[3][j]);
+      }
+    }
+  }
+  const int j0 = c * LG_C + 4 * tx;
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    float lo[4], hi[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) f2_unpack(acc[p][j], lo[j], hi[j]);
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int r = rq * LG_C + 8 * ty + 2 * p + u;
+      if (r >= Tm) continue;
+      float* dst = lg + (h * Tm + r) * Tn + j0;
+      const float* v = u ? hi : lo;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (j0 + j < Tn) dst[j] = v[j] * inv_sqrt_d;
     }
   }
 }
@@ -594,7 +632,7 @@ __global__ void __launch_bounds__(256) csc_kernel(const uint32_t* __restrict__ b
 // ---------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------
-int kbar_cols(int Tn) { return (Tn + 3) & ~3; }
+int kbar_chunks(int Tn) { return (Tn + LG_C - 1) / LG_C; }
 
 template <int E>
 static cudaError_t launch_select_t(const float* lg, int BH, int Tm, int Tn, int W, int K, unsigned long long thr,
@@ -615,30 +653,41 @@ static cudaError_t launch_select_e(const float* lg, int BH, int Tm, int Tn, int 
 }
 
 template <int D>
-static cudaError_t launch_logits_d(const float* qbar, const float* kbT, float* lg, int BH, int Tm, int Tn,
-                                   cudaStream_t s) {
+static cudaError_t launch_logits_d(const float* qbar, const float* kbc, float* lg, int BH, int Tm, int Tn, int* status,
+                                   unsigned long long wait_limit_ns, cudaStream_t s) {
+  constexpr int kMaxDev = 64;
+  static bool attr_set[kMaxDev] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  if (dev < 0 || dev >= kMaxDev || !attr_set[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(logits_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               LogitSmem<D>::TOTAL);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < kMaxDev) attr_set[dev] = true;
+  }
   KernelTimer kt(KID_LOGITS, s);
-  return launch_k(logits_kernel<D>, dim3((Tn + LG_KEYS - 1) / LG_KEYS, (Tm + LG_ROWS - 1) / LG_ROWS, BH), dim3(256),
-                  0, s, true, qbar, kbT, lg, Tm, Tn, kbar_cols(Tn), 1.0f / sqrtf((float)D));
+  return launch_k(logits_kernel<D>, dim3(kbar_chunks(Tn), kbar_chunks(Tm), BH), dim3(128),
+                  (size_t)LogitSmem<D>::TOTAL, s, true, qbar, kbc, lg, Tm, Tn, 1.0f / sqrtf((float)D), status,
+                  wait_limit_ns);
 }
 
 template <int D>
-static cudaError_t launch_pool_d(const void* q, const void* k, float* qbar, float* kbT, int BH, int N, int Tm, int Tn,
+static cudaError_t launch_pool_d(const void* q, const void* k, float* qbar, float* kbc, int BH, int N, int Tm, int Tn,
                                  int bq, int bkv, cudaStream_t s) {
   KernelTimer kt(KID_POOL, s);
   return launch_k(pool_kernel<D>, dim3(Tm + Tn, BH), dim3(256), 0, s, false, static_cast<const __nv_bfloat16*>(q),
-                  static_cast<const __nv_bfloat16*>(k), qbar, kbT, N, Tm, Tn, kbar_cols(Tn), bq, bkv);
+                  static_cast<const __nv_bfloat16*>(k), qbar, kbc, N, Tm, Tn, bq, bkv);
 }
 
-cudaError_t launch_mask(const void* q, const void* k, float* qbar, float* kbT, float* lg, int BH, int N, int d,
+cudaError_t launch_mask(const void* q, const void* k, float* qbar, float* kbc, float* lg, int BH, int N, int d,
                         int Tm, int Tn, int bq, int bkv, int K, unsigned long long thr, const MaskOut& out,
                         int* col_cnt, int* col_idx, uint32_t* bits, int W, int* status,
                         unsigned long long wait_limit_ns, cudaStream_t s) {
-  (void)wait_limit_ns;
-  cudaError_t e = d == 128 ? launch_pool_d<128>(q, k, qbar, kbT, BH, N, Tm, Tn, bq, bkv, s)
-                           : launch_pool_d<64>(q, k, qbar, kbT, BH, N, Tm, Tn, bq, bkv, s);
+  cudaError_t e = d == 128 ? launch_pool_d<128>(q, k, qbar, kbc, BH, N, Tm, Tn, bq, bkv, s)
+                           : launch_pool_d<64>(q, k, qbar, kbc, BH, N, Tm, Tn, bq, bkv, s);
   if (e != cudaSuccess) return e;
-  e = d == 128 ? launch_logits_d<128>(qbar, kbT, lg, BH, Tm, Tn, s) : launch_logits_d<64>(qbar, kbT, lg, BH, Tm, Tn, s);
+  e = d == 128 ? launch_logits_d<128>(qbar, kbc, lg, BH, Tm, Tn, status, wait_limit_ns, s)
+               : launch_logits_d<64>(qbar, kbc, lg, BH, Tm, Tn, status, wait_limit_ns, s);
   if (e != cudaSuccess) return e;
   e = launch_select_e(lg, BH, Tm, Tn, W, K, thr, out, bits, status, s);
   if (e != cudaSuccess) return e;
