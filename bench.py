@@ -128,8 +128,8 @@ def kernel_work(name, B, H, N, d, Tm, Tn, kept, fwd_flops):
         return "hbm", 4.0 * B * H * Tm * ((Tn + 31) // 32) + 4.0 * (kept + B * H * Tn), "byte"
     if name == "v_to_f16_kernel":
         return "hbm", 4.0 * e, "byte"
-    if name == "bwd_pre_kernel":
-        return "hbm", 20.0 * e + 4.0 * B * H * N, "byte"
+    if name == "bwd_pre_kernel":     # O, O_lo, dO, Q read; fp16 dO, Q and D written
+        return "hbm", 12.0 * e + 4.0 * B * H * N, "byte"
     return None, 0.0, None
 
 

@@ -209,15 +209,15 @@ SPA2_API spa2_status spa2_sparse_attn_fwd(const void* q, const void* k, const vo
  *   dS_ij = P_ij * (dP_ij - D_i),  dQ_i = sum_j dS_ij K_j * scale,
  *   dK_j = sum_i dS_ij^T Q_i * scale.
  * The mask is held constant (no gradient through pooling or selection).
- * Precision: the dK/dV pass runs every product on fp16 copies of Q, K, V and
+ * Precision: the dK/dV pass runs every product on fp16 values of Q, K, V and
  * dO (bf16 -> fp16 is exact for magnitudes in [2^-14, 65504]; smaller ones
  * round to fp16 subnormals, absolute error <= 2^-25): S = Q K^T, dP = dO V^T,
  * and P (in [0, 1]) and dS enter dV = P^T dO and dK = dS^T Q as fp16. The dQ
- * pass recomputes S from the bf16 inputs and dP from the fp16 copies, and dS
- * enters dQ = dS K as a hi + lo pair of bf16 values (about 16 significant
- * bits). Accumulation is fp32 throughout and D uses o + o_lo when o_lo is
- * given. Q, K, V or dO of magnitude > 65504 is clamped for the fp16 copies
- * and reported as SPA2_ERR_RANGE.
+ * pass recomputes S and dP from the bf16 inputs, and dS enters dQ = dS K as
+ * a hi + lo pair of bf16 values (about 16 significant bits). Accumulation is
+ * fp32 throughout and D uses o + o_lo when o_lo is given. Q, K, V or dO of
+ * magnitude > 65504 is clamped for the fp16 values and reported as
+ * SPA2_ERR_RANGE.
  * dK and dV are accumulated per kv-block (CSC column), dQ per q-block (CSR
  * row, recomputing S and dP), so no output is accumulated atomically and the
  * results are deterministic.
@@ -230,8 +230,8 @@ SPA2_API spa2_status spa2_sparse_attn_fwd(const void* q, const void* k, const vo
  *   dq, dk, dv       : [B, H, N, d] device outputs of type grad_dtype
  *   grad_dtype       : SPA2_DTYPE_BF16 or SPA2_DTYPE_F32
  *   ws               : spa2_workspace_bytes(SPA2_OP_BWD, ...) bytes (holds D,
- *                      the fp16 copies of dO, V, Q and K, and the tile lists
- *                      for sizes other than (128, 64))
+ *                      fp16 copies of dO and Q, and the tile lists for sizes
+ *                      other than (128, 64))
  */
 SPA2_API spa2_status spa2_sparse_attn_bwd(const void* q, const void* k, const void* v, const void* o,
                                           const void* o_lo, const float* lse, const void* dout, int B, int H, int N,

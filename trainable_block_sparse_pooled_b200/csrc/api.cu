@@ -125,9 +125,7 @@ struct BwdWs {
   int* status;
   float* dvec;
   void* do16;
-  void* v16;
   void* q16;
-  void* k16;
   TileWs tiles;
   size_t bytes;
 };
@@ -140,11 +138,7 @@ static BwdWs bwd_ws(void* ws, const Shape& s) {
   off += al256((size_t)s.BH * s.N * 4);
   w.do16 = base + off;
   off += al256((size_t)s.BH * s.N * s.d * 2);
-  w.v16 = base + off;
-  off += al256((size_t)s.BH * s.N * s.d * 2);
   w.q16 = base + off;
-  off += al256((size_t)s.BH * s.N * s.d * 2);
-  w.k16 = base + off;
   off += al256((size_t)s.BH * s.N * s.d * 2);
   w.bytes = tile_ws(base, off, s, true, &w.tiles);
   return w;
@@ -411,10 +405,10 @@ spa2_status spa2_sparse_attn_bwd(const void* q, const void* k, const void* v, co
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)d);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const bool f32 = grad_dtype == SPA2_DTYPE_F32;
-  CUtensorMap tq, tk, tv, tdo, tq16, tk16, tdq;
-  if (!make_map(&tq, q, s, 128) || !make_map(&tk, k, s, 64) || !make_map(&tv, w.v16, s, 64, true) ||
+  CUtensorMap tq, tk, tv, tdo, tq16, tdq;
+  if (!make_map(&tq, q, s, 128) || !make_map(&tk, k, s, 64) || !make_map(&tv, v, s, 64) ||
       !make_map(&tdo, w.do16, s, 128, true) || !make_map(&tq16, w.q16, s, 128, true) ||
-      !make_map(&tk16, w.k16, s, 64, true) || !(f32 ? make_map_f32(&tdq, dq, s, 128) : make_map(&tdq, dq, s, 128)))
+      !(f32 ? make_map_f32(&tdq, dq, s, 128) : make_map(&tdq, dq, s, 128)))
     return SPA2_ERR_CUDA;
   SPA2_CUDA_TRY(cudaMemsetAsync(w.status, 0, 4, st));
   const int *rc = mask->row_cnt, *ri = mask->row_idx, *cc = mask->col_cnt, *ci = mask->col_idx;
@@ -427,8 +421,8 @@ spa2_status spa2_sparse_attn_bwd(const void* q, const void* k, const void* v, co
     cc = w.tiles.csc_cnt;
     ci = w.tiles.csc_idx;
   }
-  BwdArgs a{&tq, &tk, &tv, &tdo, &tq16, &tk16, &tdq, q, k, o, o_lo, dout, v, lse, rc, ri, cc, ci, w.dvec, w.do16,
-            w.v16, w.q16, w.k16, dq, dk, dv, f32 ? 1 : 0, (int)s.BH, s.N, s.TMt, s.TNt, scale,
+  BwdArgs a{&tq, &tk, &tv, &tdo, &tq16, &tdq, q, k, o, o_lo, dout, v, lse, rc, ri, cc, ci, w.dvec, w.do16,
+            w.q16, dq, dk, dv, f32 ? 1 : 0, (int)s.BH, s.N, s.TMt, s.TNt, scale,
             scale * 1.4426950408889634f, w.status, g_wait_limit_ns, s.tiled ? 1 : 0};
   SPA2_CUDA_TRY(launch_bwd(a, d, st));
   return SPA2_OK;

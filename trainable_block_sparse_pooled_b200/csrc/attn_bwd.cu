@@ -5,9 +5,10 @@
 //   dV_j += P^T dO_i      dP = dO_i V_j^T      dS = P * (dP - D_i)
 //   dQ_i += dS K_j * sc   dK_j += dS^T Q_i * sc,  D_i = rowsum(dO_i * O_i).
 //
-// bwd_pre_kernel   D = rowsum(dO * (O + O_lo)) in fp32, and fp16 copies of dO,
-//                  V, Q and K for the fp16 products below (|x| > 65504 is clamped
-//                  and reported as SPA2_ERR_RANGE).
+// bwd_pre_kernel   D = rowsum(dO * (O + O_lo)) in fp32, and fp16 copies of dO
+//                  and Q, the tiles the dK/dV pass streams for its fp16
+//                  products (|x| > 65504 is clamped and reported as
+//                  SPA2_ERR_RANGE).
 // bwd_dkdv_kernel  one CTA per (kv-block j, head), looping over the q-blocks i
 //                  that keep j (CSC column of j), accumulating dV_j and dK_j in
 //                  TMEM (tcgen05 MMAs, fp32 accumulation):
@@ -15,7 +16,10 @@
 //                    dP  = dO_i V_j^T   fp16  M=128 (q) N=64 (kv) K=d    A,B K-major
 //                    dV^T += dO_i^T P   fp16  M=d       N=64 (kv) K=128  A,B MN-major
 //                    dK^T += Q_i^T dS   fp16  M=d       N=64 (kv) K=128  A,B MN-major
-//                  (fp16 copies of Q, K, V, dO). Warps 0-7 turn S, dP into P and
+//                  (fp16 copies of Q and dO from the pre-pass; K_j and V_j, which
+//                  stay in shared memory for the whole column, arrive as bf16
+//                  and warps 0-7 convert them there, with the same clamp and
+//                  report, before the first product). Warps 0-7 turn S, dP into P and
 //                  dS as fp16 tiles (11-bit significands; an fp16 dS keeps dK
 //                  within a few 1e-3 of the float64 result on the sink-key cases,
 //                  where a bf16 dS does not); warpgroup h handles kv columns
@@ -24,7 +28,8 @@
 //                  the tensor pipe runs dV/dK(t). Warp 8: TMA producer; warp 9:
 //                  MMA issuer, issuing whichever product is ready.
 // bwd_dq_kernel    one CTA per (q-block i, head), looping over the kv-blocks j
-//                  that i keeps (CSR row of i); recomputes S and dP, forms dS as a
+//                  that i keeps (CSR row of i); recomputes S and dP (bf16
+//                  operands as given: Q, dO in TMEM, K, V streamed), forms dS as a
 //                  hi + lo pair of bf16 values (about 16 significant bits: dQ is
 //                  the gradient most sensitive to dS rounding) and accumulates
 //                  dQ_i = sum_j dS_ij K_j in TMEM
@@ -60,7 +65,7 @@ struct BwdSmem {
   alignas(1024) uint8_t dO[2][CH][128 * 128];    // dO_i fp16
   alignas(1024) uint8_t p[2][128 * 128];         // P  [128 q][64 kv] fp16, tile t in buffer t mod 2
   alignas(1024) uint8_t ds[2][128 * 128];        // dS [128 q][64 kv] fp16
-  uint64_t kv_full;
+  uint64_t kv_full, kv_conv;
   uint64_t qd_full[2], qd_empty[2], sdp_full[2];
   uint64_t pds_full[2], pds_empty[2], acc_done, drain;
   uint32_t tmem_base;
@@ -85,8 +90,8 @@ SPA2_DEV void split_bf16(float a, float b, uint32_t& hi, uint32_t& lo) {
 // TILED: list entries may carry exclusion bits (block sizes other than (128, 64))
 template <int D, bool TILED>
 __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q16,
-                                                                  const __grid_constant__ CUtensorMap tm_k16,
-                                                                  const __grid_constant__ CUtensorMap tm_v16,
+                                                                  const __grid_constant__ CUtensorMap tm_k,
+                                                                  const __grid_constant__ CUtensorMap tm_v,
                                                                   const __grid_constant__ CUtensorMap tm_do16,
                                                                   const float* __restrict__ lse,
                                                              const float* __restrict__ dvec,
@@ -96,7 +101,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
                                                              float scale, float scale_log2, int* status,
                                                              unsigned long long wait_limit_ns) {
   constexpr int CH = D / 64;
-  // every product of this kernel takes fp16 operands (fp16 copies of Q, K, V, dO)
+  // every product of this kernel takes fp16 operands (Q, dO copies; K, V converted here)
   constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, false, false, /*f16=*/true);
   constexpr uint32_t IDESC_DP = IDESC_S;
   constexpr uint32_t IDESC_T = idesc_bf16_f32(128, 64, true, true, /*f16=*/true);  // dV^T and dK^T
@@ -123,6 +128,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
   }
   if (threadIdx.x == 256) {
     mbar_init(&sm.kv_full, 1);
+    mbar_init(&sm.kv_conv, 256);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.qd_full[s], 1);
       mbar_init(&sm.qd_empty[s], 1);
@@ -154,13 +160,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
     // ---------------- TMA producer ----------------
     if (lane == 0 && n > 0) {
       tma_prefetch_desc(&tm_q16);
-      tma_prefetch_desc(&tm_k16);
-      tma_prefetch_desc(&tm_v16);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do16);
       mbar_expect_tx(&sm.kv_full, 2 * KV_BYTES);
       for (int c = 0; c < CH; ++c) {
-        tma_load_3d(sm.k[c], &tm_k16, &sm.kv_full, c * 64, j * 64, bh);
-        tma_load_3d(sm.v[c], &tm_v16, &sm.kv_full, c * 64, j * 64, bh);
+        tma_load_3d(sm.k[c], &tm_k, &sm.kv_full, c * 64, j * 64, bh);
+        tma_load_3d(sm.v[c], &tm_v, &sm.kv_full, c * 64, j * 64, bh);
       }
       int issued = 0;
       for (int t = 0; t < n; ++t) {
@@ -228,7 +234,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
       // S/dP goes first, so the P / dS warps work on tile U+1 while the tensor
       // pipe runs dV/dK(U).
       int T = 0, U = 0;  // S/dP and dV/dK products issued
-      bool ok = wait_bar_all(&sm.kv_full, 0, wc);
+      bool ok = wait_bar_all(&sm.kv_conv, 0, wc);  // K_j, V_j in shared memory as fp16
       uint64_t t0 = 0;
       uint32_t idle = 0;
       while (ok && U < n) {
@@ -265,6 +271,34 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
     const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const uint64_t scale2 = f2_pack(scale_log2, scale_log2);
     bool ok = true;
+    if (n > 0) {
+      // K_j, V_j (bf16, swizzled as loaded) -> fp16 in place, 16 bytes per step
+      ok = wait_warp(&sm.kv_full, 0, wc);
+      if (ok) {
+        bool bad = false;
+        constexpr int UNITS = CH * 64 * 128 / 16;  // 16-byte units of one tensor
+#pragma unroll 1
+        for (int x = (int)threadIdx.x; x < 2 * UNITS; x += 256) {
+          uint4* u = reinterpret_cast<uint4*>(x < UNITS ? &sm.k[0][0] : &sm.v[0][0]) + (x % UNITS);
+          uint4 w = *u;
+          uint32_t* e = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&e[c]));
+            if (!(fabsf(f.x) <= 65504.f) || !(fabsf(f.y) <= 65504.f)) {
+              bad = true;
+              f.x = fminf(fmaxf(f.x, -65504.f), 65504.f);
+              f.y = fminf(fmaxf(f.y, -65504.f), 65504.f);
+            }
+            e[c] = pack_f16(f.x, f.y);
+          }
+          *u = w;
+        }
+        if (bad) report(status, SPA2_ERR_RANGE);
+      }
+      fence_proxy_async_smem();  // the tensor core reads what these generic stores wrote
+      mbar_arrive(&sm.kv_conv);
+    }
     // lse / D of the next tile's row, loaded a tile ahead
     float lse_n = INFINITY, d_n = 0.f;
     if (n > 0) {
@@ -398,7 +432,7 @@ template <int D>
 struct DqSmem {
   static constexpr int CH = D / 64;
   alignas(1024) uint8_t k[DQ_KS][CH][64 * 128];    // K_j bf16
-  alignas(1024) uint8_t v[DQ_KS][CH][64 * 128];    // V_j fp16
+  alignas(1024) uint8_t v[DQ_KS][CH][64 * 128];    // V_j bf16
   uint64_t qd_ready;
   uint64_t kv_full[DQ_KS], kv_empty[DQ_KS];
   uint64_t sdp_full[2], ds_full[2];
@@ -419,10 +453,10 @@ struct DqSmem {
 // 64b+32h .. +15 / +16 .. +31), dP[b] 128+64b, dQ 256 .. 256+d, Q 384, dO 448.
 template <int D, bool TILED>
 __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_k,
-                                                               const __grid_constant__ CUtensorMap tm_v16,
+                                                               const __grid_constant__ CUtensorMap tm_v,
                                                                const __grid_constant__ CUtensorMap tm_dq,
                                                                const __nv_bfloat16* __restrict__ qg,
-                                                               const __half* __restrict__ do16,
+                                                               const __nv_bfloat16* __restrict__ dout,
                                                                const float* __restrict__ lse,
                                                                const float* __restrict__ dvec,
                                                                const int* __restrict__ row_cnt,
@@ -432,7 +466,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_cons
                                                                unsigned long long wait_limit_ns) {
   constexpr int CH = D / 64;
   constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, false, false);
-  constexpr uint32_t IDESC_DP = idesc_bf16_f32(128, 64, false, false, /*f16=*/true);
+  constexpr uint32_t IDESC_DP = IDESC_S;
   constexpr uint32_t IDESC_Q = idesc_bf16_f32(128, D, false, true);
   constexpr uint32_t KV_BYTES = 64 * D * 2;
   constexpr uint32_t T_S = 0, T_DP = 128, T_DQ = 256, T_Q = 384, T_DO = 448;
@@ -486,7 +520,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_cons
     // ---------------- TMA producer: the K / V ring ----------------
     if (lane == 0 && n > 0) {
       tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v16);
+      tma_prefetch_desc(&tm_v);
       int issued = 0;
       for (int t = 0; t < n; ++t) {
         const int slot = t % DQ_KS;
@@ -500,7 +534,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_cons
         mbar_expect_tx(&sm.kv_full[slot], 2 * KV_BYTES);
         for (int c = 0; c < CH; ++c) {
           tma_load_3d(sm.k[slot][c], &tm_k, &sm.kv_full[slot], c * 64, j * 64, bh);
-          tma_load_3d(sm.v[slot][c], &tm_v16, &sm.kv_full[slot], c * 64, j * 64, bh);
+          tma_load_3d(sm.v[slot][c], &tm_v, &sm.kv_full[slot], c * 64, j * 64, bh);
         }
         issued = t + 1;
       }
@@ -561,7 +595,7 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_cons
     // Q_i (warpgroup 0) and dO_i (warpgroup 1) into TMEM, one row per thread
     {
       const uint4* src = h == 0 ? reinterpret_cast<const uint4*>(qg + ((long long)bh * N + row) * D)
-                                : reinterpret_cast<const uint4*>(do16 + ((long long)bh * N + row) * D);
+                                : reinterpret_cast<const uint4*>(dout + ((long long)bh * N + row) * D);
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
         uint32_t w[32];
@@ -680,18 +714,15 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_cons
   }
 }
 
-// D = rowsum(dO * (O + O_lo)) in fp32; fp16 copies of the dO, V, Q and K rows
+// D = rowsum(dO * (O + O_lo)) in fp32; fp16 copies of the dO and Q rows
 // (|x| > 65504 clamped and reported). D / 8 threads per row, 16-byte accesses.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
                                                       const __nv_bfloat16* __restrict__ o_lo,
                                                       const __nv_bfloat16* __restrict__ dout,
-                                                      const __nv_bfloat16* __restrict__ v,
                                                       const __nv_bfloat16* __restrict__ q,
-                                                      const __nv_bfloat16* __restrict__ k,
                                                       float* __restrict__ dvec, uint32_t* __restrict__ do16,
-                                                      uint32_t* __restrict__ v16, uint32_t* __restrict__ q16,
-                                                      uint32_t* __restrict__ k16, long long rows, int* status) {
+                                                      uint32_t* __restrict__ q16, long long rows, int* status) {
   // one 16-byte access per tensor per thread (every tensor is 16-byte aligned
   // and rows are D * 2 bytes): D / 8 threads per row, 8 elements each
   constexpr int TPR = D / 8;
@@ -704,16 +735,12 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __res
     const uint4 ow = *reinterpret_cast<const uint4*>(o + off);
     const uint4 lw = o_lo ? *reinterpret_cast<const uint4*>(o_lo + off) : make_uint4(0u, 0u, 0u, 0u);
     const uint4 bw = *reinterpret_cast<const uint4*>(dout + off);
-    const uint4 vw = *reinterpret_cast<const uint4*>(v + off);
     const uint4 qw = *reinterpret_cast<const uint4*>(q + off);
-    const uint4 kw = *reinterpret_cast<const uint4*>(k + off);
     const uint32_t* O = reinterpret_cast<const uint32_t*>(&ow);
     const uint32_t* L = reinterpret_cast<const uint32_t*>(&lw);
     const uint32_t* Bd = reinterpret_cast<const uint32_t*>(&bw);
-    const uint32_t* Vv = reinterpret_cast<const uint32_t*>(&vw);
     const uint32_t* Qq = reinterpret_cast<const uint32_t*>(&qw);
-    const uint32_t* Kk = reinterpret_cast<const uint32_t*>(&kw);
-    uint32_t d16[4], v16w[4], q16w[4], k16w[4];
+    uint32_t d16[4], q16w[4];
     auto f2 = [](uint32_t w) { return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w)); };
     // fp16 copy of a bf16 pair; |x| > 65504 (or NaN) is clamped and flagged
     auto to16 = [&bad](float2 x) {
@@ -734,15 +761,11 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __res
       acc = fmaf(a.x, b.x, acc);
       acc = fmaf(a.y, b.y, acc);
       d16[e] = to16(b);
-      v16w[e] = to16(f2(Vv[e]));
       q16w[e] = to16(f2(Qq[e]));
-      k16w[e] = to16(f2(Kk[e]));
     }
     const long long w = off / 2;  // 32-bit word of the fp16 copies
     *reinterpret_cast<uint4*>(do16 + w) = make_uint4(d16[0], d16[1], d16[2], d16[3]);
-    *reinterpret_cast<uint4*>(v16 + w) = make_uint4(v16w[0], v16w[1], v16w[2], v16w[3]);
     *reinterpret_cast<uint4*>(q16 + w) = make_uint4(q16w[0], q16w[1], q16w[2], q16w[3]);
-    *reinterpret_cast<uint4*>(k16 + w) = make_uint4(k16w[0], k16w[1], k16w[2], k16w[3]);
   }
 #pragma unroll
   for (int s = TPR / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffff, acc, s);
@@ -753,14 +776,13 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __res
 template <int D, bool TILED>
 static cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
   const long long rows = (long long)a.BH * a.N;
-  // 1. D and the fp16 copies of dO and V
+  // 1. D and the fp16 copies of dO and Q
   constexpr int PRE_ROWS = 256 / (D / 8);  // rows per 256-thread block
   {
     KernelTimer kt(KID_BWD_PRE, s);
     bwd_pre_kernel<D><<<(unsigned)((rows + PRE_ROWS - 1) / PRE_ROWS), 256, 0, s>>>(
       (const __nv_bfloat16*)a.o, (const __nv_bfloat16*)a.o_lo, (const __nv_bfloat16*)a.dout,
-      (const __nv_bfloat16*)a.v, (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, a.dvec, (uint32_t*)a.do16,
-      (uint32_t*)a.v16, (uint32_t*)a.q16, (uint32_t*)a.k16, rows, a.status);
+      (const __nv_bfloat16*)a.q, a.dvec, (uint32_t*)a.do16, (uint32_t*)a.q16, rows, a.status);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -771,7 +793,7 @@ static cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     KernelTimer kt(KID_BWD_DKDV, s);
     bwd_dkdv_kernel<D, TILED><<<dim3(a.Tn, a.BH), BWD_THREADS, smem, s>>>(
-        *a.tm_q16, *a.tm_k16, *a.tm_v, *a.tm_do, a.lse, a.dvec, a.col_cnt, a.col_idx, a.dk, a.dv, a.grad_f32, a.N, a.Tm,
+        *a.tm_q16, *a.tm_k, *a.tm_v, *a.tm_do, a.lse, a.dvec, a.col_cnt, a.col_idx, a.dk, a.dv, a.grad_f32, a.N, a.Tm,
         a.Tn, a.scale, a.scale_log2, a.status, a.wait_limit_ns);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -783,7 +805,7 @@ static cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     KernelTimer kt(KID_BWD_DQ, s);
     bwd_dq_kernel<D, TILED><<<dim3(a.Tm, a.BH), DQ_THREADS, smem, s>>>(
-        *a.tm_k, *a.tm_v, *a.tm_dq, static_cast<const __nv_bfloat16*>(a.q), static_cast<const __half*>(a.do16),
+        *a.tm_k, *a.tm_v, *a.tm_dq, static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.dout),
         a.lse, a.dvec, a.row_cnt, a.row_idx, a.grad_f32, a.N, a.Tm, a.Tn, a.scale, a.scale_log2, a.status,
         a.wait_limit_ns);
     e = cudaGetLastError();

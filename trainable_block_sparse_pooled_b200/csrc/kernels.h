@@ -83,10 +83,9 @@ cudaError_t launch_v_to_f16(const void* v, void* v16, long long elems, int* stat
 struct BwdArgs {
   const CUtensorMap* tm_q;    // Q bf16, box {64, 128, 1}
   const CUtensorMap* tm_k;    // K bf16, box {64, 64, 1}
-  const CUtensorMap* tm_v;    // fp16 copy of V, box {64, 64, 1}
+  const CUtensorMap* tm_v;    // V bf16, box {64, 64, 1}
   const CUtensorMap* tm_do;   // fp16 copy of dO, box {64, 128, 1}
   const CUtensorMap* tm_q16;  // fp16 copy of Q, box {64, 128, 1}
-  const CUtensorMap* tm_k16;  // fp16 copy of K, box {64, 64, 1}
   const CUtensorMap* tm_dq;   // dQ output: fp32 box {32, 128, 1} or bf16 box {64, 128, 1}, 128-byte swizzle
   const void* q;
   const void* k;
@@ -101,9 +100,7 @@ struct BwdArgs {
   const int* col_idx;
   float* dvec;     // [BH, N]
   void* do16;      // [BH, N, d] fp16
-  void* v16;       // [BH, N, d] fp16
   void* q16;       // [BH, N, d] fp16
-  void* k16;       // [BH, N, d] fp16
   void* dq;
   void* dk;
   void* dv;
