@@ -410,7 +410,7 @@ spa2_status spa2_sparse_attn_bwd(const void* q, const void* k, const void* v, co
       !make_map(&tdo, w.do16, s, 128, true) || !make_map(&tq16, w.q16, s, 128, true) ||
       !(f32 ? make_map_f32(&tdq, dq, s, 128) : make_map(&tdq, dq, s, 128)))
     return SPA2_ERR_CUDA;
-  SPA2_CUDA_TRY(cudaMemsetAsync(w.status, 0, 4, st));
+  SPA2_CUDA_TRY(cudaMemsetAsync(w.status, 0, 256, st));  // status word and the dK/dV column ticket
   const int *rc = mask->row_cnt, *ri = mask->row_idx, *cc = mask->col_cnt, *ci = mask->col_idx;
   if (s.tiled) {
     SPA2_CUDA_TRY(launch_tile_lists(mask->row_cnt, mask->row_idx, mask->col_cnt, mask->col_idx, (int)s.BH, s.Tm, s.Tn,
@@ -423,7 +423,7 @@ spa2_status spa2_sparse_attn_bwd(const void* q, const void* k, const void* v, co
   }
   BwdArgs a{&tq, &tk, &tv, &tdo, &tq16, &tdq, q, k, o, o_lo, dout, v, lse, rc, ri, cc, ci, w.dvec, w.do16,
             w.q16, dq, dk, dv, f32 ? 1 : 0, (int)s.BH, s.N, s.TMt, s.TNt, scale,
-            scale * 1.4426950408889634f, w.status, g_wait_limit_ns, s.tiled ? 1 : 0};
+            scale * 1.4426950408889634f, w.status, w.status + 32, g_wait_limit_ns, s.tiled ? 1 : 0};
   SPA2_CUDA_TRY(launch_bwd(a, d, st));
   return SPA2_OK;
 }

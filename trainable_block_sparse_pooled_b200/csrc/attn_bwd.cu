@@ -65,9 +65,10 @@ struct BwdSmem {
   alignas(1024) uint8_t dO[2][CH][128 * 128];    // dO_i fp16
   alignas(1024) uint8_t p[2][128 * 128];         // P  [128 q][64 kv] fp16, tile t in buffer t mod 2
   alignas(1024) uint8_t ds[2][128 * 128];        // dS [128 q][64 kv] fp16
-  uint64_t kv_full, kv_conv;
+  uint64_t kv_full, kv_conv, kv_empty;
   uint64_t qd_full[2], qd_empty[2], sdp_full[2];
-  uint64_t pds_full[2], pds_empty[2], acc_done, drain;
+  uint64_t pds_full[2], pds_empty[2], acc_done[2], drain;
+  int col_j[2], col_bh[2], col_n[2];  // the columns the producer has started, slot = column count mod 2
   uint32_t tmem_base;
   int abort_flag;
   int never;
@@ -87,19 +88,29 @@ SPA2_DEV void split_bf16(float a, float b, uint32_t& hi, uint32_t& lo) {
 
 }  // namespace
 
-// TILED: list entries may carry exclusion bits (block sizes other than (128, 64))
+// TILED: list entries may carry exclusion bits (block sizes other than (128, 64)).
+// Persistent: one CTA per SM takes kv columns (j, head) from an atomic ticket
+// (ticket: an int the launch's caller zeroes) until total_cols are done. The
+// Q / dO ring, the S / dP and P / dS buffers run on per-CTA tile counters that
+// continue across columns; dV^T / dK^T alternate between two TMEM sets, so the
+// previous column's gradients are written (by warps 0-7, after they have
+// converted the next column's K_j / V_j) while the tensor pipe starts on the
+// next column, and the next K_j / V_j is loaded as soon as the last S / dP of
+// the current column has run.
 template <int D, bool TILED>
 __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q16,
                                                                   const __grid_constant__ CUtensorMap tm_k,
                                                                   const __grid_constant__ CUtensorMap tm_v,
                                                                   const __grid_constant__ CUtensorMap tm_do16,
                                                                   const float* __restrict__ lse,
-                                                             const float* __restrict__ dvec,
-                                                             const int* __restrict__ col_cnt,
-                                                             const int* __restrict__ col_idx, void* __restrict__ dk,
-                                                             void* __restrict__ dv, int grad_f32, int N, int Tm, int Tn,
-                                                             float scale, float scale_log2, int* status,
-                                                             unsigned long long wait_limit_ns) {
+                                                                  const float* __restrict__ dvec,
+                                                                  const int* __restrict__ col_cnt,
+                                                                  const int* __restrict__ col_idx,
+                                                                  void* __restrict__ dk, void* __restrict__ dv,
+                                                                  int grad_f32, int N, int Tm, int Tn, int total_cols,
+                                                                  int* __restrict__ ticket, float scale,
+                                                                  float scale_log2, int* status,
+                                                                  unsigned long long wait_limit_ns) {
   constexpr int CH = D / 64;
   // every product of this kernel takes fp16 operands (Q, dO copies; K, V converted here)
   constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, false, false, /*f16=*/true);
@@ -109,18 +120,15 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
   constexpr uint32_t KV_BYTES = 64 * D * 2;
   // MN-major A operand (dO^T, Q^T): stride between the two 64-row halves of M = d
   constexpr uint32_t LBO_DT = (D == 128) ? 128 * 128 : 0;
-  constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 320;
+  constexpr uint32_t T_S = 0, T_DP = 128, T_ACC = 256;  // dV^T at T_ACC + 128 set, dK^T 64 columns after
   constexpr float LOG2E = 1.4426950408889634f;
+  constexpr int END = -2;  // column slot value: no more columns
 
   extern __shared__ uint8_t smem_raw[];
   BwdSmem<D>& sm = *reinterpret_cast<BwdSmem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
   const int warp = __shfl_sync(0xffffffffu, (int)(threadIdx.x >> 5), 0);  // warp-uniform
   const uint32_t lane = lane_id();
-  const int j = blockIdx.x;
-  const int bh = blockIdx.y;
-  const long long colid = (long long)bh * Tn + j;
-  const int kv_valid = min(64, N - j * 64);
 
   if (warp == 9) {
     tmem_alloc(&sm.tmem_base, 512);
@@ -129,14 +137,15 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
   if (threadIdx.x == 256) {
     mbar_init(&sm.kv_full, 1);
     mbar_init(&sm.kv_conv, 256);
+    mbar_init(&sm.kv_empty, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.qd_full[s], 1);
       mbar_init(&sm.qd_empty[s], 1);
       mbar_init(&sm.sdp_full[s], 1);
       mbar_init(&sm.pds_full[s], 256);
       mbar_init(&sm.pds_empty[s], 1);
+      mbar_init(&sm.acc_done[s], 1);
     }
-    mbar_init(&sm.acc_done, 1);
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     sm.never = 0;
@@ -149,101 +158,141 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
   const WaitCtx wc{&sm.abort_flag, status, wait_limit_ns};
   const WaitCtx drain_wc{&sm.never, nullptr, wait_limit_ns};
 
-  int n = __shfl_sync(0xffffffffu, col_cnt[colid], 0);  // warp-uniform
-  if (n < 0 || n > Tm) {
-    if (threadIdx.x == 0) report(status, SPA2_ERR_DEVICE_BOUNDS);
-    n = -1;  // error: write nothing
-  }
-  const int* q_list = col_idx + colid * Tm;
-
   if (warp == 8) {
-    // ---------------- TMA producer ----------------
-    if (lane == 0 && n > 0) {
+    // ---------------- TMA producer: per column K_j, V_j, then its Q / dO tiles ----------------
+    if (lane == 0) {
       tma_prefetch_desc(&tm_q16);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do16);
-      mbar_expect_tx(&sm.kv_full, 2 * KV_BYTES);
-      for (int c = 0; c < CH; ++c) {
-        tma_load_3d(sm.k[c], &tm_k, &sm.kv_full, c * 64, j * 64, bh);
-        tma_load_3d(sm.v[c], &tm_v, &sm.kv_full, c * 64, j * 64, bh);
-      }
-      int issued = 0;
-      for (int t = 0; t < n; ++t) {
-        const int s = t & 1;
-        if (t >= 2 && !wait_bar(&sm.qd_empty[s], ((t >> 1) - 1) & 1, wc)) break;
-        const int i = q_list[t] & TILE_ID_MASK;
-        if (i >= Tm) {
-          report(status, SPA2_ERR_DEVICE_BOUNDS);
-          sm.abort_flag = 1;
+      int g = 0;           // Q / dO tiles issued by this CTA
+      bool ok = true;
+      int c = 0;
+      for (;; ++c) {
+        // the K / V buffer is free once every S / dP of the previous column has run
+        if (c >= 1 && !wait_bar(&sm.kv_empty, (c - 1) & 1, wc)) ok = false;
+        const int cidx = ok ? atomicAdd(ticket, 1) : total_cols;
+        if (cidx >= total_cols) {
+          sm.col_n[c & 1] = END;
+          mbar_arrive(&sm.kv_full);
           break;
         }
-        mbar_expect_tx(&sm.qd_full[s], 2 * QT_BYTES);
-        for (int c = 0; c < CH; ++c) {
-          tma_load_3d(sm.q[s][c], &tm_q16, &sm.qd_full[s], c * 64, i * 128, bh);
-          tma_load_3d(sm.dO[s][c], &tm_do16, &sm.qd_full[s], c * 64, i * 128, bh);
+        const int j = cidx % Tn, bh = cidx / Tn;
+        int n = col_cnt[cidx];
+        if (n < 0 || n > Tm) {
+          report(status, SPA2_ERR_DEVICE_BOUNDS);
+          n = -1;  // error: this column writes nothing
         }
-        issued = t + 1;
+        sm.col_j[c & 1] = j;
+        sm.col_bh[c & 1] = bh;
+        sm.col_n[c & 1] = n;
+        if (n > 0) {
+          mbar_expect_tx(&sm.kv_full, 2 * KV_BYTES);
+          for (int cc = 0; cc < CH; ++cc) {
+            tma_load_3d(sm.k[cc], &tm_k, &sm.kv_full, cc * 64, j * 64, bh);
+            tma_load_3d(sm.v[cc], &tm_v, &sm.kv_full, cc * 64, j * 64, bh);
+          }
+        } else {
+          mbar_arrive(&sm.kv_full);
+        }
+        const int* q_list = col_idx + (long long)cidx * Tm;
+        for (int t = 0; t < n && ok; ++t, ++g) {
+          const int s = g & 1;
+          if (g >= 2 && !wait_bar(&sm.qd_empty[s], ((g >> 1) - 1) & 1, wc)) {
+            ok = false;
+            break;
+          }
+          const int i = q_list[t] & TILE_ID_MASK;
+          if (i >= Tm) {
+            report(status, SPA2_ERR_DEVICE_BOUNDS);
+            sm.abort_flag = 1;
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&sm.qd_full[s], 2 * QT_BYTES);
+          for (int cc = 0; cc < CH; ++cc) {
+            tma_load_3d(sm.q[s][cc], &tm_q16, &sm.qd_full[s], cc * 64, i * 128, bh);
+            tma_load_3d(sm.dO[s][cc], &tm_do16, &sm.qd_full[s], cc * 64, i * 128, bh);
+          }
+        }
+        if (!ok) {
+          sm.col_n[(c + 1) & 1] = END;  // lets the others leave once they see the next column
+          break;
+        }
       }
-      for (int t = max(0, issued - 2); t < issued; ++t) wait_bar(&sm.qd_full[t & 1], (t >> 1) & 1, drain_wc);
-      wait_bar(&sm.kv_full, 0, drain_wc);
+      // no copy may still be landing when the CTA exits
+      for (int t = max(0, g - 2); t < g; ++t) wait_bar(&sm.qd_full[t & 1], (t >> 1) & 1, drain_wc);
+      wait_bar(&sm.kv_full, c & 1, drain_wc);
     }
   } else if (warp == 9) {
     // ---------------- MMA issuer ----------------
-    if (n > 0) {  // all 32 lanes; elect.sync picks the issuing lane
-      const uint32_t p_addr = smem_u32(sm.p[0]), ds_addr = smem_u32(sm.ds[0]);
-      // S(t), dP(t) into TMEM buffer t mod 2 (Q / dO stage t mod 2)
-      auto issue_sdp = [&](int t) {
-        const int s = t & 1;
-        tc_fence_after();
+    const uint32_t p_addr = smem_u32(sm.p[0]), ds_addr = smem_u32(sm.ds[0]);
+    // S(g), dP(g) into TMEM buffer g mod 2 (Q / dO stage g mod 2)
+    auto issue_sdp = [&](int g) {
+      const int s = g & 1;
+      tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (64 * 128) + (kk & 3) * 32;
-          const uint32_t offq = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-          mma_ss_el(tmem + T_S + s * 64, sdesc_sw128(smem_u32(sm.q[s][0]) + offq, 16, 1024),
-                    sdesc_sw128(smem_u32(sm.k[0]) + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
-        }
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * (64 * 128) + (kk & 3) * 32;
+        const uint32_t offq = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+        mma_ss_el(tmem + T_S + s * 64, sdesc_sw128(smem_u32(sm.q[s][0]) + offq, 16, 1024),
+                  sdesc_sw128(smem_u32(sm.k[0]) + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+      }
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (64 * 128) + (kk & 3) * 32;
-          const uint32_t offq = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-          mma_ss_el(tmem + T_DP + s * 64, sdesc_sw128(smem_u32(sm.dO[s][0]) + offq, 16, 1024),
-                    sdesc_sw128(smem_u32(sm.v[0]) + off, 16, 1024), IDESC_DP, kk > 0 ? 1u : 0u);
-        }
-        mma_commit_el(&sm.sdp_full[s]);
-      };
-      // dV^T += dO^T P; dK^T += Q^T dS (fp16); K = 128 query rows
-      auto issue_dvdk = [&](int u) {
-        const int su = u & 1;
-        const uint32_t pb = (uint32_t)su * (128 * 128);
-        tc_fence_after();
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * (64 * 128) + (kk & 3) * 32;
+        const uint32_t offq = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+        mma_ss_el(tmem + T_DP + s * 64, sdesc_sw128(smem_u32(sm.dO[s][0]) + offq, 16, 1024),
+                  sdesc_sw128(smem_u32(sm.v[0]) + off, 16, 1024), IDESC_DP, kk > 0 ? 1u : 0u);
+      }
+      mma_commit_el(&sm.sdp_full[s]);
+    };
+    // dV^T += dO^T P; dK^T += Q^T dS (fp16); K = 128 query rows; first = first tile of the column
+    auto issue_dvdk = [&](int g, uint32_t acc, bool first) {
+      const int su = g & 1;
+      const uint32_t pb = (uint32_t)su * (128 * 128);
+      tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss_el(tmem + T_DV, sdesc_sw128(smem_u32(sm.dO[su][0]) + kk * 2048, LBO_DT, 1024),
-                    sdesc_sw128(p_addr + pb + kk * 2048, 0, 1024), IDESC_T, (u > 0 || kk > 0) ? 1u : 0u);
+      for (int kk = 0; kk < 8; ++kk)
+        mma_ss_el(tmem + acc, sdesc_sw128(smem_u32(sm.dO[su][0]) + kk * 2048, LBO_DT, 1024),
+                  sdesc_sw128(p_addr + pb + kk * 2048, 0, 1024), IDESC_T, (!first || kk > 0) ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss_el(tmem + T_DK, sdesc_sw128(smem_u32(sm.q[su][0]) + kk * 2048, LBO_DT, 1024),
-                    sdesc_sw128(ds_addr + pb + kk * 2048, 0, 1024), IDESC_T, (u > 0 || kk > 0) ? 1u : 0u);
-        mma_commit_el(&sm.qd_empty[su]);
-        mma_commit_el(&sm.pds_empty[su]);
-      };
+      for (int kk = 0; kk < 8; ++kk)
+        mma_ss_el(tmem + acc + 64, sdesc_sw128(smem_u32(sm.q[su][0]) + kk * 2048, LBO_DT, 1024),
+                  sdesc_sw128(ds_addr + pb + kk * 2048, 0, 1024), IDESC_T, (!first || kk > 0) ? 1u : 0u);
+      mma_commit_el(&sm.qd_empty[su]);
+      mma_commit_el(&sm.pds_empty[su]);
+    };
+    int g0 = 0;  // first tile of the current column (per-CTA count)
+    int cv = 0;  // columns with tiles so far: the accumulator set is cv mod 2
+    bool ok = true;
+    for (int c = 0; ok; ++c) {
+      if (!wait_bar_all(&sm.kv_conv, c & 1, wc)) break;  // K_j, V_j in shared memory as fp16
+      const int n = sm.col_n[c & 1];
+      if (n == END) break;
+      if (n <= 0) {
+        mma_commit_el(&sm.kv_empty);
+        continue;
+      }
+      const uint32_t acc = T_ACC + (uint32_t)(cv & 1) * 128;
       // Issue whichever product is ready. S/dP(T) needs its Q / dO tile and
       // dV/dK(T-2) issued (the P / dS warps are then done reading TMEM buffer
       // T mod 2); dV/dK(U) needs the P / dS tile of U. Of two ready products
       // S/dP goes first, so the P / dS warps work on tile U+1 while the tensor
       // pipe runs dV/dK(U).
-      int T = 0, U = 0;  // S/dP and dV/dK products issued
-      bool ok = wait_bar_all(&sm.kv_conv, 0, wc);  // K_j, V_j in shared memory as fp16
+      int T = 0, U = 0;  // S/dP and dV/dK products issued in this column
       uint64_t t0 = 0;
       uint32_t idle = 0;
-      while (ok && U < n) {
-        if (T < n && T <= U + 1 && test_wait_all(&sm.qd_full[T & 1], (T >> 1) & 1)) {
-          issue_sdp(T++);
+      while (U < n) {
+        const int gT = g0 + T, gU = g0 + U;
+        if (T < n && T <= U + 1 && test_wait_all(&sm.qd_full[gT & 1], (gT >> 1) & 1)) {
+          issue_sdp(gT);
+          if (++T == n) mma_commit_el(&sm.kv_empty);  // K_j / V_j no longer read
           idle = 0;
           t0 = 0;
-        } else if (U < T && test_wait_all(&sm.pds_full[U & 1], (U >> 1) & 1)) {
-          issue_dvdk(U++);
+        } else if (U < T && test_wait_all(&sm.pds_full[gU & 1], (gU >> 1) & 1)) {
+          issue_dvdk(gU, acc, U == 0);
+          ++U;
           idle = 0;
           t0 = 0;
         } else if ((++idle & 63u) == 0u) {
@@ -257,24 +306,75 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
               *wc.abort_flag = 1;
             }
             ok = false;
+            break;
           }
         }
       }
-      if (ok) mma_commit_el(&sm.acc_done);
-      mma_commit_el(&sm.drain);
-      wait_bar_all(&sm.drain, 0, drain_wc);
+      if (ok) mma_commit_el(&sm.acc_done[cv & 1]);
+      g0 += n;
+      ++cv;
     }
+    mma_commit_el(&sm.drain);
+    wait_bar_all(&sm.drain, 0, drain_wc);
   } else {
-    // ---------------- P / dS warps 0-7 ----------------
+    // ---------------- P / dS warps 0-7; gradient epilogue ----------------
     const int h = warp >> 2;           // kv columns 32h .. 32h+31
     const int r = threadIdx.x & 127;   // query row == TMEM lane
     const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const uint64_t scale2 = f2_pack(scale_log2, scale_log2);
     bool ok = true;
-    if (n > 0) {
-      // K_j, V_j (bf16, swizzled as loaded) -> fp16 in place, 16 bytes per step
-      ok = wait_warp(&sm.kv_full, 0, wc);
-      if (ok) {
+    int g0 = 0;                               // first tile of the current column (per-CTA count)
+    int cv = 0;                               // columns with tiles so far (accumulator set cv mod 2)
+    int prev_n = END, prev_j = 0, prev_bh = 0;  // the column whose gradients are still in TMEM
+    // gradients of column (j, bh) from TMEM set `set` (or zeros when no q-block keeps it):
+    // warpgroup 0 writes dV_j = (dV^T)^T, warpgroup 1 dK_j = scale * (dK^T)^T; thread r <-> feature r
+    auto epilogue = [&](int n, int j, int bh, int set) {
+      const int kv_valid = min(64, N - j * 64);
+      const long long base = ((long long)bh * N + (long long)j * 64) * D + r;
+      void* dst = h == 0 ? dv : dk;
+      if (n == 0) {
+        if (r < D) {
+          for (int c = 0; c < kv_valid; ++c) {
+            if (grad_f32)
+              static_cast<float*>(dst)[base + (long long)c * D] = 0.f;
+            else
+              static_cast<__nv_bfloat16*>(dst)[base + (long long)c * D] = __float2bfloat16(0.f);
+          }
+        }
+        return;
+      }
+      if (n < 0 || !ok) return;
+      tc_fence_after();
+      uint32_t a[32], b[32];
+      const uint32_t col = T_ACC + (uint32_t)set * 128 + (h == 0 ? 0 : 64);
+      tmem_ld32(tl + col, a);
+      tmem_ld32(tl + col + 32, b);
+      tmem_wait_ld();
+      const float f = h == 0 ? 1.f : scale;
+      if (r < D) {
+        if (grad_f32) {
+          float* o = static_cast<float*>(dst) + base;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            if (c < kv_valid) o[(long long)c * D] = __uint_as_float(a[c]) * f;
+            if (c + 32 < kv_valid) o[(long long)(c + 32) * D] = __uint_as_float(b[c]) * f;
+          }
+        } else {
+          __nv_bfloat16* o = static_cast<__nv_bfloat16*>(dst) + base;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            if (c < kv_valid) o[(long long)c * D] = __float2bfloat16(__uint_as_float(a[c]) * f);
+            if (c + 32 < kv_valid) o[(long long)(c + 32) * D] = __float2bfloat16(__uint_as_float(b[c]) * f);
+          }
+        }
+      }
+    };
+    for (int c = 0;; ++c) {
+      if (!wait_warp(&sm.kv_full, c & 1, wc)) ok = false;
+      const int n = ok ? sm.col_n[c & 1] : END;
+      const int j = sm.col_j[c & 1], bh = sm.col_bh[c & 1];
+      if (n > 0) {
+        // K_j, V_j (bf16, swizzled as loaded) -> fp16 in place, 16 bytes per step
         bool bad = false;
         constexpr int UNITS = CH * 64 * 128 / 16;  // 16-byte units of one tensor
 #pragma unroll 1
@@ -283,134 +383,113 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
           uint4 w = *u;
           uint32_t* e = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&e[c]));
+          for (int q2 = 0; q2 < 4; ++q2) {
+            float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&e[q2]));
             if (!(fabsf(f.x) <= 65504.f) || !(fabsf(f.y) <= 65504.f)) {
               bad = true;
               f.x = fminf(fmaxf(f.x, -65504.f), 65504.f);
               f.y = fminf(fmaxf(f.y, -65504.f), 65504.f);
             }
-            e[c] = pack_f16(f.x, f.y);
+            e[q2] = pack_f16(f.x, f.y);
           }
           *u = w;
         }
         if (bad) report(status, SPA2_ERR_RANGE);
+        fence_proxy_async_smem();  // the tensor core reads what these generic stores wrote
       }
-      fence_proxy_async_smem();  // the tensor core reads what these generic stores wrote
       mbar_arrive(&sm.kv_conv);
-    }
-    // lse / D of the next tile's row, loaded a tile ahead
-    float lse_n = INFINITY, d_n = 0.f;
-    if (n > 0) {
-      const long long row = (long long)(q_list[0] & TILE_ID_MASK) * 128 + r;
-      if (row < N) {
-        lse_n = lse[(long long)bh * N + row];
-        d_n = dvec[(long long)bh * N + row];
-      }
-    }
-    for (int t = 0; t < n; ++t) {
-      const int s = t & 1;
-      const float nlse2 = -lse_n * LOG2E, Dr = d_n;
-      if (t + 1 < n) {
-        const long long row = (long long)(q_list[t + 1] & TILE_ID_MASK) * 128 + r;
-        lse_n = row < N ? lse[(long long)bh * N + row] : INFINITY;
-        d_n = row < N ? dvec[(long long)bh * N + row] : 0.f;
-      }
-      if (!wait_warp(&sm.sdp_full[s], (t >> 1) & 1, wc)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      // P / dS buffer t mod 2 must have been consumed by dV/dK(t-2)
-      if (t >= 2 && !wait_warp(&sm.pds_empty[s], ((t >> 1) - 1) & 1, wc)) {
-        ok = false;
-        break;
-      }
-      const uint64_t nlse2x2 = f2_pack(nlse2, nlse2), d2 = f2_pack(Dr, Dr);
-      // this row's half excluded (a 64-row query block that does not keep kv tile j)
-      const bool excl = TILED && tile_excluded(q_list[t], r >> 6);
-#pragma unroll
-      for (int sub = 0; sub < 2; ++sub) {
-        const int c0 = h * 32 + sub * 16;  // first kv column of this 16-column slice
-        uint32_t sa[16], pa[16];
-        tmem_ld16(tl + T_S + s * 64 + c0, sa);
-        tmem_ld16(tl + T_DP + s * 64 + c0, pa);
-        tmem_wait_ld();
-        uint32_t pk[8], dk16[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sa[2 * e]), __uint_as_float(sa[2 * e + 1])), scale2,
-                                     nlse2x2);
-          float x0, x1;
-          f2_unpack(x2, x0, x1);
-          float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-          if (kv_valid < 64) {  // ragged last kv-block only
-            if (c0 + 2 * e >= kv_valid) p0 = 0.f;
-            if (c0 + 2 * e + 1 >= kv_valid) p1 = 0.f;
-          }
-          if (excl) p0 = p1 = 0.f;
-          pk[e] = pack_f16(p0, p1);
-          const uint64_t ds2 = f2_mul(f2_pack(p0, p1),
-                                      f2_sub(f2_pack(__uint_as_float(pa[2 * e]), __uint_as_float(pa[2 * e + 1])), d2));
-          float s0, s1;
-          f2_unpack(ds2, s0, s1);
-          dk16[e] = pack_f16(s0, s1);
-        }
-        const uint32_t u0 = c0 >> 3;  // 16-byte unit of the slice's first column
-#pragma unroll
-        for (int w = 0; w < 2; ++w) {
-          const uint32_t off = sw128_offset(r, u0 + w);
-          *reinterpret_cast<uint4*>(sm.p[s] + off) =
-              make_uint4(pk[4 * w], pk[4 * w + 1], pk[4 * w + 2], pk[4 * w + 3]);
-          *reinterpret_cast<uint4*>(sm.ds[s] + off) =
-              make_uint4(dk16[4 * w], dk16[4 * w + 1], dk16[4 * w + 2], dk16[4 * w + 3]);
+      // the previous column's gradients, while the tensor pipe starts on this one
+      if (prev_n != END) {
+        if (prev_n > 0) {
+          const int pv = cv - 1;  // its accumulator use
+          if (ok) ok = wait_warp(&sm.acc_done[pv & 1], (pv >> 1) & 1, wc);
+          epilogue(prev_n, prev_j, prev_bh, pv & 1);
+        } else {
+          epilogue(prev_n, prev_j, prev_bh, 0);
         }
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(&sm.pds_full[s]);
-    }
-    // epilogue: warpgroup 0 writes dV_j = (dV^T)^T, warpgroup 1 dK_j = scale * (dK^T)^T;
-    // thread r <-> feature r
-    const long long base = ((long long)bh * N + (long long)j * 64) * D + r;
-    void* dst = h == 0 ? dv : dk;
-    if (n == 0) {
-      // no q-block keeps kv-block j: its gradients are zero
-      if (r < D) {
-        for (int c = 0; c < kv_valid; ++c) {
-          if (grad_f32)
-            static_cast<float*>(dst)[base + (long long)c * D] = 0.f;
-          else
-            static_cast<__nv_bfloat16*>(dst)[base + (long long)c * D] = __float2bfloat16(0.f);
+      if (n == END) break;
+      prev_n = n;
+      prev_j = j;
+      prev_bh = bh;
+      if (n <= 0) continue;
+      ++cv;  // this column accumulates into set (cv - 1) mod 2
+      const int* q_list = col_idx + ((long long)bh * Tn + j) * Tm;
+      const int kv_valid = min(64, N - j * 64);
+      // lse / D of the next tile's row, loaded a tile ahead
+      float lse_n = INFINITY, d_n = 0.f;
+      {
+        const long long row = (long long)(q_list[0] & TILE_ID_MASK) * 128 + r;
+        if (row < N) {
+          lse_n = lse[(long long)bh * N + row];
+          d_n = dvec[(long long)bh * N + row];
         }
       }
-    } else if (n > 0) {
-      if (ok) ok = wait_warp(&sm.acc_done, 0, wc);
-      if (ok) {
+      for (int t = 0; t < n; ++t) {
+        const int g = g0 + t, s = g & 1;
+        const float nlse2 = -lse_n * LOG2E, Dr = d_n;
+        if (t + 1 < n) {
+          const long long row = (long long)(q_list[t + 1] & TILE_ID_MASK) * 128 + r;
+          lse_n = row < N ? lse[(long long)bh * N + row] : INFINITY;
+          d_n = row < N ? dvec[(long long)bh * N + row] : 0.f;
+        }
+        if (!wait_warp(&sm.sdp_full[s], (g >> 1) & 1, wc)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        uint32_t a[32], b[32];
-        const uint32_t col = h == 0 ? T_DV : T_DK;
-        tmem_ld32(tl + col, a);
-        tmem_ld32(tl + col + 32, b);
-        tmem_wait_ld();
-        const float f = h == 0 ? 1.f : scale;
-        if (r < D) {
-          if (grad_f32) {
-            float* o = static_cast<float*>(dst) + base;
+        // P / dS buffer g mod 2 must have been consumed by dV/dK(g-2)
+        if (g >= 2 && !wait_warp(&sm.pds_empty[s], ((g >> 1) - 1) & 1, wc)) {
+          ok = false;
+          break;
+        }
+        const uint64_t nlse2x2 = f2_pack(nlse2, nlse2), d2 = f2_pack(Dr, Dr);
+        // this row's half excluded (a 64-row query block that does not keep kv tile j)
+        const bool excl = TILED && tile_excluded(q_list[t], r >> 6);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              if (c < kv_valid) o[(long long)c * D] = __uint_as_float(a[c]) * f;
-              if (c + 32 < kv_valid) o[(long long)(c + 32) * D] = __uint_as_float(b[c]) * f;
-            }
-          } else {
-            __nv_bfloat16* o = static_cast<__nv_bfloat16*>(dst) + base;
+        for (int sub = 0; sub < 2; ++sub) {
+          const int c0 = h * 32 + sub * 16;  // first kv column of this 16-column slice
+          uint32_t sa[16], pa[16];
+          tmem_ld16(tl + T_S + s * 64 + c0, sa);
+          tmem_ld16(tl + T_DP + s * 64 + c0, pa);
+          tmem_wait_ld();
+          uint32_t pk[8], dk16[8];
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              if (c < kv_valid) o[(long long)c * D] = __float2bfloat16(__uint_as_float(a[c]) * f);
-              if (c + 32 < kv_valid) o[(long long)(c + 32) * D] = __float2bfloat16(__uint_as_float(b[c]) * f);
+          for (int e = 0; e < 8; ++e) {
+            const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sa[2 * e]), __uint_as_float(sa[2 * e + 1])), scale2,
+                                       nlse2x2);
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+            if (kv_valid < 64) {  // ragged last kv-block only
+              if (c0 + 2 * e >= kv_valid) p0 = 0.f;
+              if (c0 + 2 * e + 1 >= kv_valid) p1 = 0.f;
             }
+            if (excl) p0 = p1 = 0.f;
+            pk[e] = pack_f16(p0, p1);
+            const uint64_t ds2 =
+                f2_mul(f2_pack(p0, p1), f2_sub(f2_pack(__uint_as_float(pa[2 * e]), __uint_as_float(pa[2 * e + 1])), d2));
+            float s0, s1;
+            f2_unpack(ds2, s0, s1);
+            dk16[e] = pack_f16(s0, s1);
+          }
+          const uint32_t u0 = c0 >> 3;  // 16-byte unit of the slice's first column
+#pragma unroll
+          for (int w = 0; w < 2; ++w) {
+            const uint32_t off = sw128_offset(r, u0 + w);
+            *reinterpret_cast<uint4*>(sm.p[s] + off) = make_uint4(pk[4 * w], pk[4 * w + 1], pk[4 * w + 2], pk[4 * w + 3]);
+            *reinterpret_cast<uint4*>(sm.ds[s] + off) =
+                make_uint4(dk16[4 * w], dk16[4 * w + 1], dk16[4 * w + 2], dk16[4 * w + 3]);
           }
         }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&sm.pds_full[s]);
+      }
+      g0 += n;
+      if (!ok) {
+        prev_n = -1;  // nothing to write after a failure
+        break;
       }
     }
   }
@@ -791,10 +870,14 @@ static cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
     const size_t smem = sizeof(BwdSmem<D>) + 1024;
     e = cudaFuncSetAttribute(bwd_dkdv_kernel<D, TILED>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    const int total_cols = a.BH * a.Tn;
     KernelTimer kt(KID_BWD_DKDV, s);
-    bwd_dkdv_kernel<D, TILED><<<dim3(a.Tn, a.BH), BWD_THREADS, smem, s>>>(
+    bwd_dkdv_kernel<D, TILED><<<dim3(std::min(total_cols, sms)), BWD_THREADS, smem, s>>>(
         *a.tm_q16, *a.tm_k, *a.tm_v, *a.tm_do, a.lse, a.dvec, a.col_cnt, a.col_idx, a.dk, a.dv, a.grad_f32, a.N, a.Tm,
-        a.Tn, a.scale, a.scale_log2, a.status, a.wait_limit_ns);
+        a.Tn, total_cols, a.ticket, a.scale, a.scale_log2, a.status, a.wait_limit_ns);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

@@ -109,6 +109,7 @@ struct BwdArgs {
   float scale;        // softmax_scale
   float scale_log2;   // softmax_scale * log2(e)
   int* status;
+  int* ticket;        // zero at launch: the persistent dK/dV kernel's column counter
   unsigned long long wait_limit_ns;
   int tiled;          // list entries may carry tile exclusion bits
 };
