@@ -571,7 +571,8 @@ def run_sweep(args):
     block sparsity 80 / 90 / 95 / 97% (k = (1 - target) / 2, p calibrated) and the
     k = 100% pass, at N in {8192, 32760, 65536}. One JSON line per point: mask,
     forward and backward times (CUDA events, median of --steps after --warmup),
-    sparse and dense-equivalent TFLOP/s, and speedup over the k = 100% pass."""
+    sparse and dense-equivalent TFLOP/s, and speedup over the k = 100% pass, each with
+    the SM clocks sampled (nvidia-smi) while that N's points were timed."""
     import torch
     from trainable_block_sparse_pooled_b200 import binding as b
     from trainable_block_sparse_pooled_b200 import calibrate, synth
@@ -608,6 +609,9 @@ def run_sweep(args):
             return mask.kept_blocks()
 
         points, dense_ms = [], None
+        clocks = ClockSampler(0)
+        clocks.start()
+        time.sleep(0.15)
         for target in (None, 0.80, 0.90, 0.95, 0.97):
             if target is None:
                 kf, pf = 1.0, 0.0
@@ -629,6 +633,10 @@ def run_sweep(args):
                     "fwd_dense_equiv_tflops": dense_flops / (fwd_ms * 1e-3) / 1e12,
                     "speedup_fwd": dense_ms[0] / fwd_ms, "speedup_fwd_bwd": sum(dense_ms) / (fwd_ms + bwd_ms),
                     "steps": args.steps, "warmup": args.warmup}
+            points.append(line)
+        clk = clocks.stop()
+        for line in points:
+            line["clocks"] = clk
             print(json.dumps(line), flush=True)
         del q, k, v, dout, s, mask, o, o_lo, lse, dq, dk, dv
         torch.cuda.empty_cache()
