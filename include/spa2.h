@@ -230,7 +230,8 @@ SPA2_API spa2_status spa2_sparse_attn_fwd(const void* q, const void* k, const vo
  *   dq, dk, dv       : [B, H, N, d] device outputs of type grad_dtype
  *   grad_dtype       : SPA2_DTYPE_BF16 or SPA2_DTYPE_F32
  *   ws               : spa2_workspace_bytes(SPA2_OP_BWD, ...) bytes (holds D,
- *                      fp16 copies of dO and Q, and the tile lists for sizes
+ *                      fp16 copies of dO and Q, the order in which the dK/dV
+ *                      pass takes its kv columns, and the tile lists for sizes
  *                      other than (128, 64))
  */
 SPA2_API spa2_status spa2_sparse_attn_bwd(const void* q, const void* k, const void* v, const void* o,

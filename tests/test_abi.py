@@ -40,9 +40,12 @@ def test_workspace_sizes(L):
     assert m >= 256 + B * H * (Tm + Tn) * d * 4 + B * H * Tm * 16 * 4   # Qbar, Kbar^T, kept-bit words
     assert b.spa2_workspace_bytes(b.OP_FWD, B, H, N, d) == 256 + B * H * N * d * 2   # status + fp16 V
     al = lambda n: -(-n // 256) * 256  # noqa: E731
-    # status word, D (fp32 per row), fp16 copies of dO and Q, each 256-byte aligned
-    assert b.spa2_workspace_bytes(b.OP_BWD, B, H, N, d) == 256 + al(B * H * N * 4) + 2 * al(B * H * N * d * 2)
-    assert b.spa2_workspace_bytes(b.OP_BWD, 1, 2, 1000, 64) == 256 + al(2 * 1000 * 4) + 2 * al(2 * 1000 * 64 * 2)
+    # status word, D (fp32 per row), fp16 copies of dO and Q, the order of the dK/dV
+    # pass's columns (one int per kv column), each 256-byte aligned
+    assert b.spa2_workspace_bytes(b.OP_BWD, B, H, N, d) == (256 + al(B * H * N * 4) + 2 * al(B * H * N * d * 2)
+                                                          + al(B * H * Tn * 4))
+    assert b.spa2_workspace_bytes(b.OP_BWD, 1, 2, 1000, 64) == (256 + al(2 * 1000 * 4) + 2 * al(2 * 1000 * 64 * 2)
+                                                              + al(2 * 16 * 4))
     assert b.spa2_workspace_bytes(b.OP_SELECT, 2, 3, 5, 40, 0, 0) == 256 + 256   # 2*3*5*2 words = 240 B
     # unsupported shapes report 0
     assert b.spa2_workspace_bytes(b.OP_MASK, 1, 1, 100, 96) == 0

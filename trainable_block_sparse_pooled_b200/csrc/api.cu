@@ -126,6 +126,7 @@ struct BwdWs {
   float* dvec;
   void* do16;
   void* q16;
+  int* col_order;  // the order of the dK/dV pass's columns
   TileWs tiles;
   size_t bytes;
 };
@@ -140,6 +141,8 @@ static BwdWs bwd_ws(void* ws, const Shape& s) {
   off += al256((size_t)s.BH * s.N * s.d * 2);
   w.q16 = base + off;
   off += al256((size_t)s.BH * s.N * s.d * 2);
+  w.col_order = reinterpret_cast<int*>(base + off);
+  off += al256((size_t)s.BH * s.TNt * 4);
   w.bytes = tile_ws(base, off, s, true, &w.tiles);
   return w;
 }
@@ -423,7 +426,8 @@ spa2_status spa2_sparse_attn_bwd(const void* q, const void* k, const void* v, co
   }
   BwdArgs a{&tq, &tk, &tv, &tdo, &tq16, &tdq, q, k, o, o_lo, dout, v, lse, rc, ri, cc, ci, w.dvec, w.do16,
             w.q16, dq, dk, dv, f32 ? 1 : 0, (int)s.BH, s.N, s.TMt, s.TNt, scale,
-            scale * 1.4426950408889634f, w.status, w.status + 32, g_wait_limit_ns, s.tiled ? 1 : 0};
+            scale * 1.4426950408889634f, w.status, w.status + 32, g_wait_limit_ns, s.tiled ? 1 : 0,
+            w.col_order};
   SPA2_CUDA_TRY(launch_bwd(a, d, st));
   return SPA2_OK;
 }

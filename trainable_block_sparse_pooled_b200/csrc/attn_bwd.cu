@@ -90,7 +90,9 @@ SPA2_DEV void split_bf16(float a, float b, uint32_t& hi, uint32_t& lo) {
 
 // TILED: list entries may carry exclusion bits (block sizes other than (128, 64)).
 // Persistent: one CTA per SM takes kv columns (j, head) from an atomic ticket
-// (ticket: an int the launch's caller zeroes) until total_cols are done. The
+// (ticket: an int the launch's caller zeroes) until total_cols are done, in the
+// order the pre-pass wrote to col_order (head by head, long columns first),
+// and takes its next column's ticket one column ahead (see the producer). The
 // Q / dO ring, the S / dP and P / dS buffers run on per-CTA tile counters that
 // continue across columns; dV^T / dK^T alternate between two TMEM sets, so the
 // previous column's gradients are written (by warps 0-7, after they have
@@ -106,6 +108,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
                                                                   const float* __restrict__ dvec,
                                                                   const int* __restrict__ col_cnt,
                                                                   const int* __restrict__ col_idx,
+                                                                  const int* __restrict__ col_order,
                                                                   void* __restrict__ dk, void* __restrict__ dv,
                                                                   int grad_f32, int N, int Tm, int Tn, int total_cols,
                                                                   int* __restrict__ ticket, float scale,
@@ -168,11 +171,45 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
       int g = 0;           // Q / dO tiles issued by this CTA
       bool ok = true;
       int c = 0;
+      // The next column is taken while this one runs (ticket `ahead`, column
+      // `ahead_cidx`) and its K / V are started toward L2, so the switch to it
+      // waits for an L2 copy instead of an atomic, two dependent loads and an
+      // HBM read. Not in the last round of columns, where a held ticket could
+      // leave other CTAs without work.
+      int ahead = -1, ahead_cidx = -1;
+      auto look_ahead = [&](int pos) {
+        if (ahead >= 0 || !ok || pos + (int)gridDim.x >= total_cols) return;
+        ahead = atomicAdd(ticket, 1);
+        if (ahead >= total_cols) return;
+        ahead_cidx = col_order[ahead];
+        if (ahead_cidx < 0 || ahead_cidx >= total_cols) return;  // reported when it is used
+        const int jn = ahead_cidx % Tn, bhn = ahead_cidx / Tn;
+        for (int cc = 0; cc < CH; ++cc) {
+          tma_prefetch_3d(&tm_k, cc * 64, jn * 64, bhn);
+          tma_prefetch_3d(&tm_v, cc * 64, jn * 64, bhn);
+        }
+      };
       for (;; ++c) {
         // the K / V buffer is free once every S / dP of the previous column has run
         if (c >= 1 && !wait_bar(&sm.kv_empty, (c - 1) & 1, wc)) ok = false;
-        const int cidx = ok ? atomicAdd(ticket, 1) : total_cols;
-        if (cidx >= total_cols) {
+        int pos = total_cols, cidx = -1;
+        if (ok) {
+          if (ahead >= 0) {
+            pos = ahead;
+            cidx = ahead_cidx;
+          } else {
+            pos = atomicAdd(ticket, 1);
+            if (pos < total_cols) cidx = col_order[pos];
+          }
+        }
+        ahead = -1;
+        if (pos < total_cols && (cidx < 0 || cidx >= total_cols)) {
+          report(status, SPA2_ERR_DEVICE_BOUNDS);
+          sm.abort_flag = 1;
+          ok = false;
+          pos = total_cols;
+        }
+        if (pos >= total_cols) {
           sm.col_n[c & 1] = END;
           mbar_arrive(&sm.kv_full);
           break;
@@ -198,6 +235,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
         const int* q_list = col_idx + (long long)cidx * Tm;
         for (int t = 0; t < n && ok; ++t, ++g) {
           const int s = g & 1;
+          if (t == 2) look_ahead(pos);  // the first two Q / dO tiles are on their way
           if (g >= 2 && !wait_bar(&sm.qd_empty[s], ((g >> 1) - 1) & 1, wc)) {
             ok = false;
             break;
@@ -219,6 +257,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
           sm.col_n[(c + 1) & 1] = END;  // lets the others leave once they see the next column
           break;
         }
+        look_ahead(pos);  // columns of at most two tiles
       }
       // no copy may still be landing when the CTA exits
       for (int t = max(0, g - 2); t < g; ++t) wait_bar(&sm.qd_full[t & 1], (t >> 1) & 1, drain_wc);
@@ -793,15 +832,66 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_cons
   }
 }
 
+// One head's kv columns (Tn counts from head * Tn on), longest first, written
+// as global column indices head * Tn + c: a counting sort by one 256-thread
+// block (keys clamped to [0, 1023]; the order among equal counts is whatever the
+// shared-memory atomics give, which does not matter: a column's gradients are
+// computed the same way whichever CTA takes it and whenever). The persistent
+// dK/dV pass takes its columns head by head and, within a head, long columns
+// first: it does not end on a long column, and the Q / dO tiles the running
+// columns share stay within one head's worth of L2.
+SPA2_DEV void longest_first(const int* __restrict__ cnt, int Tn, int head, int* __restrict__ order) {
+  constexpr int KEYS = 1024, PER = KEYS / 256;
+  __shared__ int start[KEYS];
+  __shared__ int warp_sum[8];
+  const int t = threadIdx.x;
+  const int* cnt_h = cnt + (long long)head * Tn;
+  int* out_h = order + (long long)head * Tn;
+  for (int k = t; k < KEYS; k += 256) start[k] = 0;
+  __syncthreads();
+  for (int c = t; c < Tn; c += 256) atomicAdd(&start[min(max(cnt_h[c], 0), KEYS - 1)], 1);
+  __syncthreads();
+  // exclusive scan in descending key order: thread t owns keys KEYS-1-PER*t ... KEYS-PER-PER*t
+  int bin[PER], sum = 0;
+#pragma unroll
+  for (int e = 0; e < PER; ++e) {
+    bin[e] = start[KEYS - 1 - PER * t - e];
+    sum += bin[e];
+  }
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if ((t & 31) >= o) incl += y;
+  }
+  if ((t & 31) == 31) warp_sum[t >> 5] = incl;
+  __syncthreads();
+  int base = incl - sum;
+  for (int w = 0; w < (t >> 5); ++w) base += warp_sum[w];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) {
+    start[KEYS - 1 - PER * t - e] = base;
+    base += bin[e];
+  }
+  __syncthreads();
+  for (int c = t; c < Tn; c += 256)
+    out_h[atomicAdd(&start[min(max(cnt_h[c], 0), KEYS - 1)], 1)] = head * Tn + c;
+  __syncthreads();  // start[] is reused by the next head of this block
+}
+
 // D = rowsum(dO * (O + O_lo)) in fp32; fp16 copies of the dO and Q rows
 // (|x| > 65504 clamped and reported). D / 8 threads per row, 16-byte accesses.
+// Blocks 0 .. BH-1 (each a stride of heads, when there are fewer blocks) also
+// write the order in which the dK/dV pass takes its columns.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
                                                       const __nv_bfloat16* __restrict__ o_lo,
                                                       const __nv_bfloat16* __restrict__ dout,
                                                       const __nv_bfloat16* __restrict__ q,
                                                       float* __restrict__ dvec, uint32_t* __restrict__ do16,
-                                                      uint32_t* __restrict__ q16, long long rows, int* status) {
+                                                      uint32_t* __restrict__ q16, long long rows,
+                                                      const int* __restrict__ col_cnt, int BH, int Tn,
+                                                      int* __restrict__ col_order, int* status) {
   // one 16-byte access per tensor per thread (every tensor is 16-byte aligned
   // and rows are D * 2 bytes): D / 8 threads per row, 8 elements each
   constexpr int TPR = D / 8;
@@ -850,6 +940,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __res
   for (int s = TPR / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffff, acc, s);
   if (row < rows && tc == 0) dvec[row] = acc;
   if (bad) report(status, SPA2_ERR_RANGE);
+  for (int head = blockIdx.x; head < BH; head += gridDim.x) longest_first(col_cnt, Tn, head, col_order);
 }
 
 template <int D, bool TILED>
@@ -861,7 +952,8 @@ static cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
     KernelTimer kt(KID_BWD_PRE, s);
     bwd_pre_kernel<D><<<(unsigned)((rows + PRE_ROWS - 1) / PRE_ROWS), 256, 0, s>>>(
       (const __nv_bfloat16*)a.o, (const __nv_bfloat16*)a.o_lo, (const __nv_bfloat16*)a.dout,
-      (const __nv_bfloat16*)a.q, a.dvec, (uint32_t*)a.do16, (uint32_t*)a.q16, rows, a.status);
+      (const __nv_bfloat16*)a.q, a.dvec, (uint32_t*)a.do16, (uint32_t*)a.q16, rows, a.col_cnt, a.BH, a.Tn, a.col_order,
+      a.status);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -876,7 +968,8 @@ static cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t s) {
     const int total_cols = a.BH * a.Tn;
     KernelTimer kt(KID_BWD_DKDV, s);
     bwd_dkdv_kernel<D, TILED><<<dim3(std::min(total_cols, sms)), BWD_THREADS, smem, s>>>(
-        *a.tm_q16, *a.tm_k, *a.tm_v, *a.tm_do, a.lse, a.dvec, a.col_cnt, a.col_idx, a.dk, a.dv, a.grad_f32, a.N, a.Tm,
+        *a.tm_q16, *a.tm_k, *a.tm_v, *a.tm_do, a.lse, a.dvec, a.col_cnt, a.col_idx, a.col_order, a.dk, a.dv,
+        a.grad_f32, a.N, a.Tm,
         a.Tn, total_cols, a.ticket, a.scale, a.scale_log2, a.status, a.wait_limit_ns);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -112,6 +112,7 @@ struct BwdArgs {
   int* ticket;        // zero at launch: the persistent dK/dV kernel's column counter
   unsigned long long wait_limit_ns;
   int tiled;          // list entries may carry tile exclusion bits
+  int* col_order;     // [BH * Tn]: the dK/dV pass's columns, head by head, long columns first (pre-pass)
 };
 cudaError_t launch_bwd(const BwdArgs& a, int d, cudaStream_t s);
 
