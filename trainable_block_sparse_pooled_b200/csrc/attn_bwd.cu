@@ -233,14 +233,21 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
           mbar_arrive(&sm.kv_full);
         }
         const int* q_list = col_idx + (long long)cidx * Tm;
+        // A stage frees when dV/dK of the tile two back has run, and the next
+        // S / dP waits for its refill: so the list entry of each tile is read
+        // before its stage is waited for, and each tile's Q / dO are prefetched
+        // into L2 when the tile before it is issued, which leaves the refill an
+        // L2 copy.
+        int i_next = n > 0 ? q_list[0] & TILE_ID_MASK : 0;
         for (int t = 0; t < n && ok; ++t, ++g) {
           const int s = g & 1;
+          const int i = i_next;
+          if (t + 1 < n) i_next = q_list[t + 1] & TILE_ID_MASK;
           if (t == 2) look_ahead(pos);  // the first two Q / dO tiles are on their way
           if (g >= 2 && !wait_bar(&sm.qd_empty[s], ((g >> 1) - 1) & 1, wc)) {
             ok = false;
             break;
           }
-          const int i = q_list[t] & TILE_ID_MASK;
           if (i >= Tm) {
             report(status, SPA2_ERR_DEVICE_BOUNDS);
             sm.abort_flag = 1;
@@ -251,6 +258,12 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
           for (int cc = 0; cc < CH; ++cc) {
             tma_load_3d(sm.q[s][cc], &tm_q16, &sm.qd_full[s], cc * 64, i * 128, bh);
             tma_load_3d(sm.dO[s][cc], &tm_do16, &sm.qd_full[s], cc * 64, i * 128, bh);
+          }
+          if (t + 1 < n && i_next < Tm) {
+            for (int cc = 0; cc < CH; ++cc) {
+              tma_prefetch_3d(&tm_q16, cc * 64, i_next * 128, bh);
+              tma_prefetch_3d(&tm_do16, cc * 64, i_next * 128, bh);
+            }
           }
         }
         if (!ok) {
