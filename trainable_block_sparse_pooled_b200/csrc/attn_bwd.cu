@@ -18,7 +18,7 @@
 //                    dK^T += Q_i^T dS   fp16  M=d       N=64 (kv) K=128  A,B MN-major
 //                  (fp16 copies of Q and dO from the pre-pass; K_j and V_j, which
 //                  stay in shared memory for the whole column, arrive as bf16
-//                  and warps 0-7 convert them there, with the same clamp and
+//                  and warps 10-13 convert them there, with the same clamp and
 //                  report, before the first product). Warps 0-7 turn S, dP into P and
 //                  dS as fp16 tiles (11-bit significands; an fp16 dS keeps dK
 //                  within a few 1e-3 of the float64 result on the sink-key cases,
@@ -26,7 +26,8 @@
 //                  32h .. 32h+31, thread = query row. P / dS tiles are
 //                  double-buffered in shared memory, so tile t+1 is formed while
 //                  the tensor pipe runs dV/dK(t). Warp 8: TMA producer; warp 9:
-//                  MMA issuer, issuing whichever product is ready.
+//                  MMA issuer, issuing whichever product is ready; warps 10-13:
+//                  the K / V conversion and the gradient epilogue of each column.
 // bwd_dq_kernel    one CTA per (q-block i, head), looping over the kv-blocks j
 //                  that i keeps (CSR row of i); recomputes S and dP (bf16
 //                  operands as given: Q, dO in TMEM, K, V streamed), forms dS as a
@@ -39,8 +40,9 @@
 //                  For d = 64 the dV^T / dK^T MMAs still run at M = 128 (the
 //                  upper 64 lanes repeat the lower ones and are ignored).
 //
-// TMEM columns (both kernels): S[2] 0..127, dP[2] 128..255; dV^T 256..319 and
-// dK^T 320..383 (dkdv), dQ 256..256+d (dq).
+// TMEM columns (both kernels): S[2] 0..127, dP[2] 128..255; dkdv: two
+// accumulator sets 256..383 and 384..511, dV^T in a set's first 64 columns and
+// dK^T in the next 64; dq: dQ 256..256+d.
 // In both kernels the MMA warp runs its issue loop with all 32 lanes and
 // elect.sync picks the lane that issues each tcgen05.mma / tcgen05.commit (the
 // descriptor arithmetic then stays on the warp-uniform datapath; a one-lane loop
@@ -54,7 +56,7 @@ namespace spa2 {
 
 namespace {
 
-constexpr int BWD_THREADS = 320;  // P/dS x 8 warps, TMA, MMA
+constexpr int BWD_THREADS = 448;  // P/dS x 8 warps, TMA, MMA, K / V conversion and gradient epilogue x 4
 
 template <int D>
 struct BwdSmem {
@@ -67,7 +69,7 @@ struct BwdSmem {
   alignas(1024) uint8_t ds[2][128 * 128];        // dS [128 q][64 kv] fp16
   uint64_t kv_full, kv_conv, kv_empty;
   uint64_t qd_full[2], qd_empty[2], sdp_full[2];
-  uint64_t pds_full[2], pds_empty[2], acc_done[2], drain;
+  uint64_t pds_full[2], pds_empty[2], acc_done[2], acc_free[2], drain;
   int col_j[2], col_bh[2], col_n[2];  // the columns the producer has started, slot = column count mod 2
   uint32_t tmem_base;
   int abort_flag;
@@ -95,10 +97,11 @@ SPA2_DEV void split_bf16(float a, float b, uint32_t& hi, uint32_t& lo) {
 // and takes its next column's ticket one column ahead (see the producer). The
 // Q / dO ring, the S / dP and P / dS buffers run on per-CTA tile counters that
 // continue across columns; dV^T / dK^T alternate between two TMEM sets, so the
-// previous column's gradients are written (by warps 0-7, after they have
-// converted the next column's K_j / V_j) while the tensor pipe starts on the
-// next column, and the next K_j / V_j is loaded as soon as the last S / dP of
-// the current column has run.
+// previous column's gradients are written (by warps 10-13, after they have
+// converted the next column's K_j / V_j) while the tensor pipe and warps 0-7
+// go on with the next column; a set's first dV/dK waits (acc_free) until its
+// gradients of two columns back have been read out. The next K_j / V_j is
+// loaded as soon as the last S / dP of the current column has run.
 template <int D, bool TILED>
 __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q16,
                                                                   const __grid_constant__ CUtensorMap tm_k,
@@ -139,7 +142,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
   }
   if (threadIdx.x == 256) {
     mbar_init(&sm.kv_full, 1);
-    mbar_init(&sm.kv_conv, 256);
+    mbar_init(&sm.kv_conv, 128);
     mbar_init(&sm.kv_empty, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.qd_full[s], 1);
@@ -148,6 +151,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
       mbar_init(&sm.pds_full[s], 256);
       mbar_init(&sm.pds_empty[s], 1);
       mbar_init(&sm.acc_done[s], 1);
+      mbar_init(&sm.acc_free[s], 128);
     }
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
@@ -327,6 +331,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
         continue;
       }
       const uint32_t acc = T_ACC + (uint32_t)(cv & 1) * 128;
+      // the set was last used two columns back: its first dV/dK here (which
+      // overwrites it) waits until warps 10-13 have read those gradients out
+      bool acc_free = cv < 2;
       // Issue whichever product is ready. S/dP(T) needs its Q / dO tile and
       // dV/dK(T-2) issued (the P / dS warps are then done reading TMEM buffer
       // T mod 2); dV/dK(U) needs the P / dS tile of U. Of two ready products
@@ -342,7 +349,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
           if (++T == n) mma_commit_el(&sm.kv_empty);  // K_j / V_j no longer read
           idle = 0;
           t0 = 0;
-        } else if (U < T && test_wait_all(&sm.pds_full[gU & 1], (gU >> 1) & 1)) {
+        } else if (U < T && (acc_free || (acc_free = test_wait_all(&sm.acc_free[cv & 1], ((cv >> 1) - 1) & 1))) &&
+                   test_wait_all(&sm.pds_full[gU & 1], (gU >> 1) & 1)) {
           issue_dvdk(gU, acc, U == 0);
           ++U;
           idle = 0;
@@ -368,55 +376,62 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
     }
     mma_commit_el(&sm.drain);
     wait_bar_all(&sm.drain, 0, drain_wc);
-  } else {
-    // ---------------- P / dS warps 0-7; gradient epilogue ----------------
-    const int h = warp >> 2;           // kv columns 32h .. 32h+31
-    const int r = threadIdx.x & 127;   // query row == TMEM lane
+  } else if (warp >= 10) {
+    // ---------------- warps 10-13: K / V to fp16, gradient epilogue ----------------
+    // Per column: convert the K_j / V_j just loaded (the next S / dP waits for
+    // it), then write the previous column's gradients from its TMEM set and
+    // release the set. Off the P / dS warps, so a column switch costs them
+    // nothing but the wait for the next S / dP.
+    const int r = (warp & 3) * 32 + (int)lane;  // TMEM lane == feature row of dV^T / dK^T
     const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    const uint64_t scale2 = f2_pack(scale_log2, scale_log2);
     bool ok = true;
-    int g0 = 0;                               // first tile of the current column (per-CTA count)
-    int cv = 0;                               // columns with tiles so far (accumulator set cv mod 2)
+    int cv = 0;                                 // columns with tiles so far (accumulator set cv mod 2)
     int prev_n = END, prev_j = 0, prev_bh = 0;  // the column whose gradients are still in TMEM
-    // gradients of column (j, bh) from TMEM set `set` (or zeros when no q-block keeps it):
-    // warpgroup 0 writes dV_j = (dV^T)^T, warpgroup 1 dK_j = scale * (dK^T)^T; thread r <-> feature r
+    // gradients of column (j, bh) from TMEM set `set` (or zeros when no q-block
+    // keeps it): dV_j = (dV^T)^T and dK_j = scale * (dK^T)^T; thread r <-> feature r
     auto epilogue = [&](int n, int j, int bh, int set) {
       const int kv_valid = min(64, N - j * 64);
       const long long base = ((long long)bh * N + (long long)j * 64) * D + r;
-      void* dst = h == 0 ? dv : dk;
       if (n == 0) {
         if (r < D) {
           for (int c = 0; c < kv_valid; ++c) {
-            if (grad_f32)
-              static_cast<float*>(dst)[base + (long long)c * D] = 0.f;
-            else
-              static_cast<__nv_bfloat16*>(dst)[base + (long long)c * D] = __float2bfloat16(0.f);
+            if (grad_f32) {
+              static_cast<float*>(dv)[base + (long long)c * D] = 0.f;
+              static_cast<float*>(dk)[base + (long long)c * D] = 0.f;
+            } else {
+              static_cast<__nv_bfloat16*>(dv)[base + (long long)c * D] = __float2bfloat16(0.f);
+              static_cast<__nv_bfloat16*>(dk)[base + (long long)c * D] = __float2bfloat16(0.f);
+            }
           }
         }
         return;
       }
       if (n < 0 || !ok) return;
       tc_fence_after();
-      uint32_t a[32], b[32];
-      const uint32_t col = T_ACC + (uint32_t)set * 128 + (h == 0 ? 0 : 64);
-      tmem_ld32(tl + col, a);
-      tmem_ld32(tl + col + 32, b);
-      tmem_wait_ld();
-      const float f = h == 0 ? 1.f : scale;
-      if (r < D) {
-        if (grad_f32) {
-          float* o = static_cast<float*>(dst) + base;
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {  // 0: dV, 1: dK
+        uint32_t a[32], b[32];
+        const uint32_t col = T_ACC + (uint32_t)set * 128 + (uint32_t)which * 64;
+        tmem_ld32(tl + col, a);
+        tmem_ld32(tl + col + 32, b);
+        tmem_wait_ld();
+        const float f = which == 0 ? 1.f : scale;
+        void* dst = which == 0 ? dv : dk;
+        if (r < D) {
+          if (grad_f32) {
+            float* o = static_cast<float*>(dst) + base;
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            if (c < kv_valid) o[(long long)c * D] = __uint_as_float(a[c]) * f;
-            if (c + 32 < kv_valid) o[(long long)(c + 32) * D] = __uint_as_float(b[c]) * f;
-          }
-        } else {
-          __nv_bfloat16* o = static_cast<__nv_bfloat16*>(dst) + base;
+            for (int c = 0; c < 32; ++c) {
+              if (c < kv_valid) o[(long long)c * D] = __uint_as_float(a[c]) * f;
+              if (c + 32 < kv_valid) o[(long long)(c + 32) * D] = __uint_as_float(b[c]) * f;
+            }
+          } else {
+            __nv_bfloat16* o = static_cast<__nv_bfloat16*>(dst) + base;
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            if (c < kv_valid) o[(long long)c * D] = __float2bfloat16(__uint_as_float(a[c]) * f);
-            if (c + 32 < kv_valid) o[(long long)(c + 32) * D] = __float2bfloat16(__uint_as_float(b[c]) * f);
+            for (int c = 0; c < 32; ++c) {
+              if (c < kv_valid) o[(long long)c * D] = __float2bfloat16(__uint_as_float(a[c]) * f);
+              if (c + 32 < kv_valid) o[(long long)(c + 32) * D] = __float2bfloat16(__uint_as_float(b[c]) * f);
+            }
           }
         }
       }
@@ -429,8 +444,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
         // K_j, V_j (bf16, swizzled as loaded) -> fp16 in place, 16 bytes per step
         bool bad = false;
         constexpr int UNITS = CH * 64 * 128 / 16;  // 16-byte units of one tensor
-#pragma unroll 1
-        for (int x = (int)threadIdx.x; x < 2 * UNITS; x += 256) {
+#pragma unroll 4
+        for (int x = (int)threadIdx.x - 320; x < 2 * UNITS; x += 128) {
           uint4* u = reinterpret_cast<uint4*>(x < UNITS ? &sm.k[0][0] : &sm.v[0][0]) + (x % UNITS);
           uint4 w = *u;
           uint32_t* e = reinterpret_cast<uint32_t*>(&w);
@@ -456,6 +471,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
           const int pv = cv - 1;  // its accumulator use
           if (ok) ok = wait_warp(&sm.acc_done[pv & 1], (pv >> 1) & 1, wc);
           epilogue(prev_n, prev_j, prev_bh, pv & 1);
+          tc_fence_before();
+          mbar_arrive(&sm.acc_free[pv & 1]);  // the set may be overwritten
         } else {
           epilogue(prev_n, prev_j, prev_bh, 0);
         }
@@ -464,8 +481,22 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
       prev_n = n;
       prev_j = j;
       prev_bh = bh;
+      if (n > 0) ++cv;  // this column accumulates into set (cv - 1) mod 2
+    }
+  } else {
+    // ---------------- P / dS warps 0-7 ----------------
+    const int h = warp >> 2;           // kv columns 32h .. 32h+31
+    const int r = threadIdx.x & 127;   // query row == TMEM lane
+    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const uint64_t scale2 = f2_pack(scale_log2, scale_log2);
+    bool ok = true;
+    int g0 = 0;  // first tile of the current column (per-CTA count)
+    for (int c = 0;; ++c) {
+      if (!wait_warp(&sm.kv_full, c & 1, wc)) ok = false;
+      const int n = ok ? sm.col_n[c & 1] : END;
+      const int j = sm.col_j[c & 1], bh = sm.col_bh[c & 1];
+      if (n == END) break;
       if (n <= 0) continue;
-      ++cv;  // this column accumulates into set (cv - 1) mod 2
       const int* q_list = col_idx + ((long long)bh * Tn + j) * Tm;
       const int kv_valid = min(64, N - j * 64);
       // lse / D of the next tile's row, loaded a tile ahead
@@ -539,10 +570,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) bwd_dkdv_kernel(const __grid_c
         mbar_arrive(&sm.pds_full[s]);
       }
       g0 += n;
-      if (!ok) {
-        prev_n = -1;  // nothing to write after a failure
-        break;
-      }
+      if (!ok) break;
     }
   }
 
