@@ -755,19 +755,21 @@ __global__ void __launch_bounds__(DQ_THREADS, 1) bwd_dq_kernel(const __grid_cons
     {
       const uint4* src = h == 0 ? reinterpret_cast<const uint4*>(qg + ((long long)bh * N + row) * D)
                                 : reinterpret_cast<const uint4*>(dout + ((long long)bh * N + row) * D);
+      // every load of the row first (one memory round trip), then the TMEM stores
+      uint32_t w[D / 64][32];
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
-        uint32_t w[32];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const uint4 x = rvalid ? src[c * 8 + e] : make_uint4(0, 0, 0, 0);
-          w[4 * e] = x.x;
-          w[4 * e + 1] = x.y;
-          w[4 * e + 2] = x.z;
-          w[4 * e + 3] = x.w;
+          w[c][4 * e] = x.x;
+          w[c][4 * e + 1] = x.y;
+          w[c][4 * e + 2] = x.z;
+          w[c][4 * e + 3] = x.w;
         }
-        tmem_st32(tl + (h == 0 ? T_Q : T_DO) + c * 32, w);
       }
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) tmem_st32(tl + (h == 0 ? T_Q : T_DO) + c * 32, w[c]);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sm.qd_ready);
