@@ -352,15 +352,27 @@ __global__ void __launch_bounds__(192, 2) fwd_kernel(const __grid_constant__ CUt
   }
 }
 
-// bf16 -> fp16 copy of V (16 bytes per thread and step); |v| > 65504 is clamped
-// to the largest finite fp16 and reported as SPA2_ERR_RANGE.
+// bf16 -> fp16 copy of V; |v| > 65504 is clamped to the largest finite fp16 and
+// reported as SPA2_ERR_RANGE. Each thread converts V16_UNROLL 16-byte units a
+// block-width apart, all of its loads issued before the first conversion, so a
+// thread keeps 64 bytes in flight (one unit at a time left the copy at ~0.8 of
+// HBM bandwidth).
+constexpr int V16_UNROLL = 4;
 __global__ void __launch_bounds__(256) v_to_f16_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
                                                        long long n8, int* status) {
   pdl_trigger();  // the forward kernel may start its prologue (Q load, TMEM, barriers)
   bool bad = false;
-  for (long long e = (long long)blockIdx.x * 256 + threadIdx.x; e < n8; e += (long long)gridDim.x * 256) {
-    const uint4 v = src[e];
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  const long long base = (long long)blockIdx.x * (256 * V16_UNROLL) + threadIdx.x;
+  uint4 v[V16_UNROLL];
+#pragma unroll
+  for (int u = 0; u < V16_UNROLL; ++u) {
+    const long long e = base + u * 256;
+    v[u] = e < n8 ? src[e] : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int u = 0; u < V16_UNROLL; ++u) {
+    const long long e = base + u * 256;
+    const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
     uint32_t o[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -372,17 +384,19 @@ __global__ void __launch_bounds__(256) v_to_f16_kernel(const uint4* __restrict__
       }
       o[i] = pack_f16(f.x, f.y);
     }
-    dst[e] = make_uint4(o[0], o[1], o[2], o[3]);
+    if (e < n8) dst[e] = make_uint4(o[0], o[1], o[2], o[3]);
   }
   if (bad) report(status, SPA2_ERR_RANGE);
 }
 
 cudaError_t launch_v_to_f16(const void* v, void* v16, long long elems, int* status, cudaStream_t s) {
   const long long n8 = elems / 8;
-  const unsigned blocks = (unsigned)((n8 + 255) / 256 < 148LL * 32 ? (n8 + 255) / 256 : 148LL * 32);
+  const long long per_block = 256LL * V16_UNROLL;
+  const long long blocks = (n8 + per_block - 1) / per_block;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   KernelTimer kt(KID_V16, s);
-  return launch_k(v_to_f16_kernel, dim3(blocks), dim3(256), 0, s, false, static_cast<const uint4*>(v),
-                  static_cast<uint4*>(v16), n8, status);
+  return launch_k(v_to_f16_kernel, dim3((unsigned)std::max(blocks, 1LL)), dim3(256), 0, s, false,
+                  static_cast<const uint4*>(v), static_cast<uint4*>(v16), n8, status);
 }
 
 template <int D, bool TILED>
