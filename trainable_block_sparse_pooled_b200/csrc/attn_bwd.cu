@@ -8,8 +8,10 @@
 // bwd_pre_kernel   D = rowsum(dO * (O + O_lo)) in fp32, and fp16 copies of dO
 //                  and Q, the tiles the dK/dV pass streams for its fp16
 //                  products (|x| > 65504 is clamped and reported as
-//                  SPA2_ERR_RANGE).
-// bwd_dkdv_kernel  one CTA per (kv-block j, head), looping over the q-blocks i
+//                  SPA2_ERR_RANGE); its first blocks also order the dK/dV
+//                  pass's columns (per head, longest first).
+// bwd_dkdv_kernel  persistent, one CTA per SM taking (kv-block j, head)
+//                  columns in turn; per column it loops over the q-blocks i
 //                  that keep j (CSC column of j), accumulating dV_j and dK_j in
 //                  TMEM (tcgen05 MMAs, fp32 accumulation):
 //                    S   = Q_i K_j^T    fp16  M=128 (q) N=64 (kv) K=d    A,B K-major
